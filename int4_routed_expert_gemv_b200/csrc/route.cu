@@ -1,0 +1,303 @@
+// Router: logits = x . W_r^T (+ bias), top-k with index tie-break, renormalised softmax
+// weights; optionally followed by the batch union in the same launch.
+//
+// The router is the first of the per-layer steps ("路由器选出专家", colibri technical
+// article "colibri 技术解读", section "引擎结构：一个 C 文件，五步 token 路径"); GLM-5.2
+// selects 8 of 256 routed experts per layer (same article, "MoE 的稀疏性").
+//
+// Logits are the double-precision sum of the exact float x float products, rounded once
+// to float.  Any summation order gives the same float except when the exact sum lies
+// within about 1e-16 (relative) of a float rounding boundary, so the selected indices
+// agree bit for bit with a sequential double-precision reference.  Selection compares
+// floats (ties, including +0 == -0, go to the lower expert index); the weights are
+// exp(l_i - l_max) / sum_j exp(l_j - l_max) over the selected logits, in double.
+#include "common.cuh"
+#include "route.cuh"
+#include "union.cuh"
+
+namespace coli {
+namespace {
+
+template <typename XT>
+__device__ __forceinline__ float4 load_x4(const XT* x, size_t i4);
+
+template <>
+__device__ __forceinline__ float4 load_x4<float>(const float* x, size_t i4)
+{
+    return __ldg(reinterpret_cast<const float4*>(x) + i4);
+}
+
+template <>
+__device__ __forceinline__ float4 load_x4<__nv_bfloat16>(const __nv_bfloat16* x, size_t i4)
+{
+    const uint2 r = __ldg(reinterpret_cast<const uint2*>(x) + i4);
+    return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                       __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ double dsum_warp(double v)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Order-preserving 64-bit key: larger value first, then smaller index.
+__device__ __forceinline__ uint64_t topk_key(float v, int e)
+{
+    uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);   // -0 and +0 compare equal
+    const uint32_t u = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+
+__device__ __forceinline__ float key_value(uint64_t key)
+{
+    const uint32_t u = (uint32_t)(key >> 32);
+    const uint32_t b = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+    return __uint_as_float(b);
+}
+
+// One warp selects the top-k of one token's logits and writes idx/w.
+__device__ void topk_warp(const float* lt, int E, int k, int32_t* idx_t, float* w_t, int lane)
+{
+    constexpr int MAXPL = kMaxExperts / 32;
+    uint64_t key[MAXPL];
+#pragma unroll
+    for (int i = 0; i < MAXPL; i++) {
+        const int e = lane + 32 * i;
+        key[i] = (e < E) ? topk_key(__ldcg(lt + e), e) : 0ull;
+    }
+    uint64_t mine = 0;   // key of slot `lane` (lanes < k)
+    for (int s = 0; s < k; s++) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < MAXPL; i++) best = key[i] > best ? key[i] : best;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+#pragma unroll
+        for (int i = 0; i < MAXPL; i++)
+            if (key[i] == best) key[i] = 0ull;   // keys are unique (index in low bits)
+        if (lane == s) mine = best;
+    }
+    const double lmax = (double)key_value(__shfl_sync(0xffffffffu, mine, 0));
+    double ex = 0.0;
+    if (lane < k) ex = exp((double)key_value(mine) - lmax);
+    const double z = dsum_warp(ex);
+    if (lane < k) {
+        idx_t[lane] = (int32_t)(0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull));
+        w_t[lane] = (float)(ex / z);
+    }
+}
+
+// Small batches: a CTA computes RB router rows for all T (<= kSmallT) tokens; threads
+// split the hidden dimension.  The last CTA to finish (ticket in the workspace header)
+// runs top-k for every token and, if asked, the batch union.
+template <typename XT, int RB>
+__global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant__ RouteParams p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ double part[8][RB * kSmallT];
+    __shared__ int is_last;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int e0 = blockIdx.x * RB;
+    const int H4 = p.H / 4;
+    const XT* x = reinterpret_cast<const XT*>(p.x);
+
+    double acc[RB][kSmallT];
+#pragma unroll
+    for (int r = 0; r < RB; r++)
+#pragma unroll
+        for (int t = 0; t < kSmallT; t++) acc[r][t] = 0.0;
+    for (int c4 = tid; c4 < H4; c4 += 256) {
+        float4 wv[RB];
+#pragma unroll
+        for (int r = 0; r < RB; r++)
+            wv[r] = (e0 + r < p.E) ? __ldcs(reinterpret_cast<const float4*>(p.w_router) +
+                                            (size_t)(e0 + r) * H4 + c4)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < kSmallT; t++) {
+            if (t < p.T) {
+                const float4 xv = load_x4<XT>(x, (size_t)t * H4 + c4);
+#pragma unroll
+                for (int r = 0; r < RB; r++) {
+                    double a = acc[r][t];
+                    a = fma((double)xv.x, (double)wv[r].x, a);
+                    a = fma((double)xv.y, (double)wv[r].y, a);
+                    a = fma((double)xv.z, (double)wv[r].z, a);
+                    a = fma((double)xv.w, (double)wv[r].w, a);
+                    acc[r][t] = a;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RB; r++)
+#pragma unroll
+        for (int t = 0; t < kSmallT; t++) {
+            const double v = dsum_warp(acc[r][t]);
+            if (lane == 0) part[warp][r * kSmallT + t] = v;
+        }
+    __syncthreads();
+    if (tid < RB * kSmallT) {
+        const int r = tid / kSmallT, t = tid % kSmallT;
+        if (t < p.T && e0 + r < p.E) {
+            double s = 0.0;
+            for (int w = 0; w < 8; w++) s += part[w][tid];
+            if (p.bias) s += (double)p.bias[e0 + r];
+            const float l = (float)s;
+            if (!isfinite(l)) set_flag(p.status, DEV_NONFINITE);
+            p.logits[(size_t)t * p.E + e0 + r] = l;
+        }
+    }
+    if (!p.do_topk) return;
+    // ---- last-CTA election: the final arrival sees every logit
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t prev = atomicAdd(&p.hdr->route_ticket, 1u);
+        is_last = (prev == gridDim.x - 1);
+        if (is_last) atomicExch(&p.hdr->route_ticket, 0u);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int t = warp; t < p.T; t += 8)
+        topk_warp(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
+                  p.w + (size_t)t * p.k, lane);
+    if (p.do_union) {
+        __threadfence();
+        __syncthreads();
+        union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status,
+                    smem);
+    }
+}
+
+// Large batches: 64 tokens x 64 experts per CTA, 32-column slabs staged in shared
+// memory, each thread accumulates 4 x 4 logits in double.
+template <typename XT>
+__global__ void __launch_bounds__(256) router_tiled_kernel(const __grid_constant__ RouteParams p)
+{
+    __shared__ float xs[32][64 + 4];
+    __shared__ float ws[32][64 + 4];
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+    const int ty = tid / 16, tx = tid % 16;
+    const XT* x = reinterpret_cast<const XT*>(p.x);
+    double acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; a++)
+#pragma unroll
+        for (int b = 0; b < 4; b++) acc[a][b] = 0.0;
+    for (int k0 = 0; k0 < p.H; k0 += 32) {
+        // 64 rows x 32 columns of x and of W_r: 512 float4 each, 2 per thread
+#pragma unroll
+        for (int q = 0; q < 2; q++) {
+            const int f = tid + 256 * q;
+            const int row = f / 8, c4 = f % 8;
+            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
+            if (t0 + row < p.T) xv = load_x4<XT>(x, ((size_t)(t0 + row) * p.H + k0) / 4 + c4);
+            if (e0 + row < p.E)
+                wv = __ldg(reinterpret_cast<const float4*>(p.w_router) +
+                           ((size_t)(e0 + row) * p.H + k0) / 4 + c4);
+            xs[c4 * 4 + 0][row] = xv.x;
+            xs[c4 * 4 + 1][row] = xv.y;
+            xs[c4 * 4 + 2][row] = xv.z;
+            xs[c4 * 4 + 3][row] = xv.w;
+            ws[c4 * 4 + 0][row] = wv.x;
+            ws[c4 * 4 + 1][row] = wv.y;
+            ws[c4 * 4 + 2][row] = wv.z;
+            ws[c4 * 4 + 3][row] = wv.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 32; kk++) {
+            const float4 a4 = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+            const float4 b4 = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+            const double a[4] = {a4.x, a4.y, a4.z, a4.w};
+            const double b[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int jj = 0; jj < 4; jj++) acc[i][jj] = fma(a[i], b[jj], acc[i][jj]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + jj;
+            if (t < p.T && e < p.E) {
+                double s = acc[i][jj];
+                if (p.bias) s += (double)p.bias[e];
+                const float l = (float)s;
+                if (!isfinite(l)) set_flag(p.status, DEV_NONFINITE);
+                p.logits[(size_t)t * p.E + e] = l;
+            }
+        }
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const __grid_constant__ RouteParams p)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t < p.T)
+        topk_warp(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
+                  p.w + (size_t)t * p.k, lane);
+}
+
+__global__ void __launch_bounds__(1024) union_kernel(const __grid_constant__ RouteParams p)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status, smem);
+}
+
+}  // namespace
+
+cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
+{
+    const bool bf16 = p.x_bf16 != 0;
+    if (p.T <= kSmallT) {
+        constexpr int RB = 2;
+        const int grid = (p.E + RB - 1) / RB;
+        size_t smem = p.do_union ? union_smem_bytes(p.E, 8) : 0;
+        auto kern = bf16 ? router_small_kernel<__nv_bfloat16, RB> : router_small_kernel<float, RB>;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<grid, 256, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    dim3 grid((p.E + 63) / 64, (p.T + 63) / 64);
+    if (bf16)
+        router_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+    else
+        router_tiled_kernel<float><<<grid, 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || !p.do_topk) return e;
+    topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !p.do_union) return e;
+    return union_launch(p, s);
+}
+
+cudaError_t union_launch(const RouteParams& p, cudaStream_t s)
+{
+    const int nt = 1024;
+    const size_t smem = union_smem_bytes(p.E, nt / 32);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    union_kernel<<<1, nt, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace coli

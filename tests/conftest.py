@@ -17,3 +17,12 @@ def pytest_configure(config):
 def cuda_available():
     import torch
     return torch.cuda.is_available()
+
+
+@pytest.fixture(scope="session")
+def colimoe():
+    """The CUDA library, built in-tree if stale (needs nvcc only, no GPU)."""
+    from int4_routed_expert_gemv_b200 import build, binding
+    build.build()
+    binding.lib()
+    return binding
