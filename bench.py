@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the routed int4 MoE layer on B200.
+
+One step = one pass of the whole hot path over one batch: route (router GEMV + top-k) and
+batch union, gate/up int4 GEMV + SwiGLU, down int4 GEMV + routing-weighted combine with
+the shared expert.  Default workload: the GLM-5.2-shaped layer decoding one token
+(hidden 6144, 256 experts of intermediate 2048, top-8 + 1 shared, fp32 activations).
+
+Timing: W untimed warm-up steps, then exactly K timed steps.  L2 is flushed (a write of
+twice its size) before every step, outside the timed intervals; each step is bracketed by
+CUDA events on the launching stream, and the kernels inside it by further events.  The
+value is tokens/s over all ranks (replicas: one independent layer per GPU), with the
+max over ranks of the summed step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; expert-weight HBM GB/s as fraction of B200 peak (decode)"
+DEFAULT_WORKLOAD = "glm52_moe_h6144_i2048_e256_k8_t1"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--pool", type=int, default=64, help="distinct token batches rotated over")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--n-experts", type=int, default=0,
+                    help="profiling captures only: keep the first N routed experts")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "gate_up": ["int4_routed_expert_gemv_b200/csrc/gemv.cu",
+                "int4_routed_expert_gemv_b200/csrc/gemv.cuh",
+                "int4_routed_expert_gemv_b200/csrc/common.cuh"],
+    "down": ["int4_routed_expert_gemv_b200/csrc/gemv.cu",
+             "int4_routed_expert_gemv_b200/csrc/gemv.cuh",
+             "int4_routed_expert_gemv_b200/csrc/common.cuh"],
+    "route_union": ["int4_routed_expert_gemv_b200/csrc/route.cu",
+                    "int4_routed_expert_gemv_b200/csrc/union.cuh"],
+}
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from an ncu capture, if the kernel is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [r for (t, r) in self.rows if t0 - 0.05 <= t <= t1 + 0.05] or [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from int4_routed_expert_gemv_b200 import binding as B
+    from int4_routed_expert_gemv_b200 import build as builder
+    from int4_routed_expert_gemv_b200 import synth
+
+    if rank == 0 or world == 1:
+        builder.build()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[args.workload]
+    if args.n_experts:
+        import dataclasses
+        shp = dataclasses.replace(wl.shape, n_experts=args.n_experts)
+        wl = dataclasses.replace(wl, shape=shp, name=f"{wl.name}_first{args.n_experts}experts")
+    if wl.layers != 1 or wl.x_dtype != "f32":
+        raise SystemExit(f"bench.py times single-layer fp32 workloads; got {wl.name}")
+    s = wl.shape
+    T = wl.tokens
+    H, I, E, k = s.hidden, s.inter, s.n_experts, s.top_k
+
+    experts = synth.experts_tensor(s, wl.seed, 0, device=dev)
+    shared = synth.shared_tensor(s, wl.seed, 0, device=dev)
+    wr = torch.from_numpy(synth.router_weight(s, wl.seed)).to(dev)
+    bias = torch.from_numpy(synth.zipf_bias(E)).to(dev) if wl.zipf else None
+    dims = B.make_dims(H, I, E, k, s.n_shared)
+    weights = B.make_weights(wr, bias, experts, shared, s.stride)
+    bufs = B.LayerBuffers(dims, T, device=dev)
+
+    R = args.pool
+    xs_host = [torch.from_numpy(synth.activations(s, wl.seed, T, 1000 + i)).pin_memory()
+               for i in range(R)]
+    xs = [x.to(dev) for x in xs_host]
+    y_host = torch.empty(T, H, dtype=torch.float32).pin_memory()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # union size of every batch in the pool (deterministic), for the byte counts
+    n_union = []
+    for i in range(R):
+        B.check(B.coli_moe_route_union(dims, wr, bias, xs[i], T, bufs.idx, bufs.w, None,
+                                       bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
+                                       bufs.ws), "route_union")
+        n_union.append(int(bufs.n_union[0].item()))
+
+    def step(i, ev=None):
+        x = xs[i % R]
+        if ev:
+            ev[0].record(stream)
+        B.check(B.coli_moe_route_union(dims, wr, bias, x, T, bufs.idx, bufs.w, None,
+                                       bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
+                                       bufs.ws), "route_union")
+        if ev:
+            ev[1].record(stream)
+        B.check(B.coli_moe_gate_up(dims, weights, x, T, bufs.union_ids, bufs.n_union,
+                                   bufs.offsets, bufs.assign, bufs.ws), "gate_up")
+        if ev:
+            ev[2].record(stream)
+        B.check(B.coli_moe_down(dims, weights, T, bufs.w, bufs.union_ids, bufs.n_union,
+                                bufs.offsets, bufs.assign, None, bufs.y, bufs.ws), "down")
+        if ev:
+            ev[3].record(stream)
+
+    def flush():
+        flush_buf.zero_()
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.2)
+    for i in range(args.warmup):
+        flush()
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    t0 = time.time()
+    for i in range(K):
+        flush()
+        step(args.warmup + i, evs[i])
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    time.sleep(0.1)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(K)])
+    step_ms = seg.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    st, bits = B.coli_moe_read_status(bufs.ws)
+    if st != B.COLI_OK:
+        raise SystemExit(f"device status {bits:#x} after the timed region")
+
+    # e2e: host buffers through the public layer call, copies inside the timed interval
+    e2e = None
+    if not args.no_e2e:
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        for i in range(min(args.warmup, 5)):
+            flush()
+            xs[0].copy_(xs_host[i % R], non_blocking=True)
+            B.check(B.coli_moe_layer(dims, weights, xs[0], T, bufs.idx, bufs.w, None,
+                                     bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
+                                     None, bufs.y, bufs.ws))
+            y_host.copy_(bufs.y[:T], non_blocking=True)
+        torch.cuda.synchronize(dev)
+        xin = torch.empty_like(xs[0])
+        for i in range(K):
+            flush()
+            ev2[i][0].record(stream)
+            xin.copy_(xs_host[i % R], non_blocking=True)
+            B.check(B.coli_moe_layer(dims, weights, xin, T, bufs.idx, bufs.w, None,
+                                     bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
+                                     None, bufs.y, bufs.ws))
+            y_host.copy_(bufs.y[:T], non_blocking=True)
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = float(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(K)))
+        e2e = (e2e_ms, T * H * 4, T * H * 4)
+
+    times = torch.tensor([total_ms, e2e[0] if e2e else 0.0], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms = float(times[0]), float(times[1])
+    if rank != 0:
+        return None
+
+    # algorithmic bytes
+    blob = s.blob_bytes
+    gu_bytes_expert = 2 * (I * H // 2) + 2 * (I * H // 64) * 2
+    dn_bytes_expert = H * I // 2 + H * (I // 64) * 2
+    nu = np.array([n_union[(args.warmup + i) % R] for i in range(K)], dtype=np.float64)
+    units = nu + s.n_shared
+    x_bytes = T * H * 4
+    h_bytes = (T * k + T * s.n_shared) * I * 4
+    route_bytes = E * H * 4 + x_bytes + T * E * 4
+    gu_bytes = units * gu_bytes_expert + x_bytes + h_bytes
+    dn_bytes = units * dn_bytes_expert + h_bytes + T * H * 4
+    step_bytes = route_bytes + units * blob + x_bytes + 2 * h_bytes + T * H * 4
+    peak, peak_kind = measured_peaks()
+    kern = {
+        "route_union": (seg[:, 0], np.full(K, route_bytes)),
+        "gate_up": (seg[:, 1], gu_bytes),
+        "down": (seg[:, 2], dn_bytes),
+    }
+    kernels = {}
+    for name, (ms, by) in kern.items():
+        avg_ms = float(ms.mean())
+        gbs = float(by.sum() / (ms.sum() * 1e-3) / 1e9)
+        kernels[name] = {"avg_us": round(avg_ms * 1e3, 3), "bytes_per_launch": float(by.mean()),
+                         "gb_s": round(gbs, 1), "frac": round(gbs / peak, 4),
+                         "share": round(float(ms.sum() / seg.sum()), 4)}
+    dom = max(kernels, key=lambda n: kernels[n]["share"])
+    traffic = recorded_traffic(dom, wl.name)
+    tokens = T * K * world
+    value = tokens / (total_ms * 1e-3)
+    launches_per_step = (1 if T <= 8 else 3) + 2
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "tokens_per_step": T, "hidden": H, "intermediate": I,
+                   "experts": E, "top_k": k, "shared_experts": s.n_shared,
+                   "weights": "gs64 int4, fp16 scales", "activations": "fp32",
+                   "l2": "flushed (2x L2 write) before every step, outside the timed intervals",
+                   "token_pool": R, "parallelism": f"replicas x{world}",
+                   "mean_union": float(nu.mean())},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gb_s"],
+                     "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "unit": "GB/s", "frac": kernels[dom]["frac"],
+                     "traffic": traffic},
+        "step_hbm": {"algorithmic_bytes": float(step_bytes.mean()),
+                     "gb_s": round(float(step_bytes.sum() / (total_ms * 1e-3) / 1e9 * world), 1),
+                     "frac_of_peak_per_gpu": round(float(step_bytes.sum() / (total_ms * 1e-3) / 1e9 / peak), 4)},
+        "kernels": kernels,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if e2e:
+        out["e2e"] = {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                      "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2],
+                      "api": "coli_moe_layer with pinned-host x in and y out"}
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    return out
+
+
+# ------------------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------
+
+def oracle_setup(wl, n_batches):
+    import oracle
+    from int4_routed_expert_gemv_b200 import synth
+    s = wl.shape
+    wr = synth.router_weight(s, wl.seed)
+    bias = synth.zipf_bias(s.n_experts) if wl.zipf else None
+    batches = []
+    blobs = {}
+    for i in range(n_batches):
+        x = synth.activations(s, wl.seed, wl.tokens, 1000 + i)
+        idx, _, _ = oracle.route(x, wr, bias, s.top_k)
+        for e in np.unique(idx):
+            if int(e) not in blobs:
+                blobs[int(e)] = synth.expert_blob(s, wl.seed, 0, int(e)).numpy()
+        batches.append(x)
+    shared = synth.expert_blob(s, wl.seed, 0, s.n_experts).numpy()
+    return wr, bias, batches, blobs, shared
+
+
+def oracle_step(wl, wr, bias, x, blobs, shared):
+    import oracle
+    s = wl.shape
+    idx, w, _ = oracle.route(x, wr, bias, s.top_k)
+    oracle.union(idx, s.n_experts)
+    sub = {int(e): blobs[int(e)] for e in np.unique(idx)}
+    return oracle.forward_sparse(s.hidden, s.inter, s.top_k, s.n_shared, x, sub, shared, idx, w)
+
+
+def cpu_baseline(wl, seconds):
+    wr, bias, batches, blobs, shared = oracle_setup(wl, 4)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle_step(wl, wr, bias, batches[n % len(batches)], blobs, shared)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 64:
+            break
+    return {"value": round(n * wl.tokens / el, 4), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{n} steps of {wl.tokens} token(s) of {wl.name} (route+union+forward, "
+                      f"scalar C, double accumulation, one thread), {el:.1f} s"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    from int4_routed_expert_gemv_b200 import synth
+    import oracle
+    oracle.build()
+    wl = synth.WORKLOADS[args.workload]
+    wr, bias, batches, blobs, shared = oracle_setup(wl, 4)
+    for i in range(args.warmup):
+        oracle_step(wl, wr, bias, batches[i % 4], blobs, shared)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(wl, wr, bias, batches[i % 4], blobs, shared)
+    el = time.perf_counter() - t0
+    v = args.steps * wl.tokens / el
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_step": wl.tokens},
+            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{args.steps} timed steps of {wl.tokens} token(s), "
+                                       "rotating over 4 token batches"},
+            "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
