@@ -173,6 +173,28 @@ COLI_API coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_we
                            int32_t* assign, const float* residual, float* y, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of coli_moe_forward for the fp32 decode path.  The colibri
+ * pages have no counterpart: this exists for callers that cannot allocate device memory
+ * or hand over a workspace -- e.g. code running inside a host framework's enqueue
+ * callback, where the framework owns all device memory and forbids new allocations, or a
+ * latency-critical loop where cudaMalloc would synchronise the device.
+ * Instead of a workspace it uses a fixed 4 MiB array in the library's device memory
+ * (present on every GPU that loads the library until the process exits).  A batch needs
+ * 256 + T * (top_k + n_shared) * inter * 4 bytes of it; larger batches return
+ * COLI_ENOMEM before anything is enqueued.  Arguments and results are those of
+ * coli_moe_forward with dtype COLI_F32.  Every call on a device shares the array and it
+ * keeps the previous call's contents (each call clears its 256-byte header and rewrites
+ * h before reading it); calls whose GPU work overlaps (e.g. on two streams) race on it,
+ * so serialise them.  The first call on a device sets up the array's device address
+ * (once per device, with that device current): make that first call before any stream
+ * capture.  Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_dims* dims,
+                                              const coli_moe_weights* weights, const float* x,
+                                              int32_t T, const float* w, const int32_t* union_ids,
+                                              const int32_t* n_union, const int32_t* offsets,
+                                              const int32_t* assign, const float* residual,
+                                              float* y, void* stream);
+
 /* RMSNorm: out [T][H] = x * gamma / sqrt(mean(x^2) + eps), computed in double and
  * rounded once to fp32.  out may alias x. */
 COLI_API coli_status coli_rmsnorm(int32_t hidden, int32_t T, const float* x, const float* gamma, double eps,

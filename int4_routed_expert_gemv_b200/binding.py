@@ -26,6 +26,7 @@ EXPORTS = [
     "coli_moe_blob_bytes", "coli_moe_workspace_bytes", "coli_moe_workspace_init",
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
     "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_rmsnorm",
+    "coli_moe_forward_noalloc",
     "coli_status_string",
 ]
 
@@ -76,6 +77,7 @@ def lib():
                 "coli_moe_down": (i32, [D, W, i32, P, P, P, P, P, P, P, P, sz, P]),
                 "coli_moe_layer": (i32, [D, W, P, i32, i32, P, P, P, P, P, P, P, P, P, P, sz, P]),
                 "coli_rmsnorm": (i32, [i32, i32, P, P, ctypes.c_double, P, P]),
+                "coli_moe_forward_noalloc": (i32, [D, W, P, i32, P, P, P, P, P, P, P, P]),
                 "coli_status_string": (ctypes.c_char_p, [i32]),
             }
             for name, (res, args) in sig.items():
@@ -185,6 +187,15 @@ def coli_moe_layer(dims, weights, x, T, idx, w, logits, union_ids, n_union, offs
                                 _p(idx), _p(w), _p(logits), _p(union_ids), _p(n_union),
                                 _p(offsets), _p(assign), _p(residual), _p(y), _p(ws),
                                 ws.numel(), _s(stream))
+
+
+def coli_moe_forward_noalloc(dims, weights, x, T, w, union_ids, n_union, offsets, assign,
+                             residual, y, stream=None) -> int:
+    """Forward without a workspace: scratch lives in a fixed 4 MiB array of the library's
+    device memory, for callers that cannot allocate (see include/colimoe.h)."""
+    return lib().coli_moe_forward_noalloc(ctypes.byref(dims), ctypes.byref(weights), _p(x), T,
+                                          _p(w), _p(union_ids), _p(n_union), _p(offsets),
+                                          _p(assign), _p(residual), _p(y), _s(stream))
 
 
 def coli_rmsnorm(hidden, T, x, gamma, eps, out, stream=None) -> int:

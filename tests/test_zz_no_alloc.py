@@ -1,0 +1,58 @@
+"""coli_moe_forward_noalloc: the forward for callers that cannot allocate device memory
+(for example code running inside a host framework's enqueue callback, where the framework
+owns all device memory, or a latency-critical loop where cudaMalloc would synchronise the
+device).  Its scratch is a fixed array in the library's device memory instead of a
+caller-owned workspace.
+
+Checked through the C ABI against the regular coli_moe_forward on the same inputs, on two
+calls in a row (the array keeps the previous call's contents), within the parity
+tolerance of the other tests.  Collected last on purpose: a run that stops at the first
+failure has run every other test before this one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from int4_routed_expert_gemv_b200 import binding as B
+from int4_routed_expert_gemv_b200 import synth
+from layers import assert_y_close, make_device_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["moe_h1024_i512_e64_k4_t4_zipf",
+                                  "glm52_moe_h6144_i2048_e256_k8_t1"])
+def test_noalloc_forward_matches_regular_forward(colimoe, name):
+    wl = synth.WORKLOADS[name]
+    L = make_device_layer(wl.shape, wl.seed, zipf=wl.zipf)
+    T = wl.tokens
+    bufs = B.LayerBuffers(L.dims, T)
+    outs = []
+    for variant in [31, 32]:                       # two calls in a row, different tokens
+        x = torch.from_numpy(synth.activations(wl.shape, wl.seed, T, variant)).cuda()
+        res = torch.from_numpy(synth.activations(wl.shape, wl.seed + 1, T, variant)).cuda()
+        B.check(B.coli_moe_route_union(L.dims, L.w_router, L.bias, x, T, bufs.idx, bufs.w,
+                                       None, bufs.union_ids, bufs.n_union, bufs.offsets,
+                                       bufs.assign, bufs.ws))
+        y_ref = torch.empty(T, wl.shape.hidden, device="cuda")
+        B.check(B.coli_moe_forward(L.dims, L.weights, x, T, bufs.idx, bufs.w, bufs.union_ids,
+                                   bufs.n_union, bufs.offsets, bufs.assign, res, y_ref, bufs.ws))
+        y = torch.full((T, wl.shape.hidden), float("nan"), device="cuda")
+        B.check(B.coli_moe_forward_noalloc(L.dims, L.weights, x, T, bufs.w, bufs.union_ids,
+                                           bufs.n_union, bufs.offsets, bufs.assign, res, y),
+                "coli_moe_forward_noalloc")
+        torch.cuda.synchronize()
+        assert_y_close(y.cpu().numpy(), y_ref.cpu().numpy())
+        outs.append(y.cpu().numpy())
+    assert not np.array_equal(outs[0], outs[1])
+
+
+def test_noalloc_rejects_batches_beyond_its_scratch(colimoe):
+    shape = synth.GLM
+    dims = B.make_dims(shape.hidden, shape.inter, shape.n_experts, shape.top_k, 1)
+    # 256 + T * 9 * 2048 * 4 bytes exceeds 4 MiB from T = 57 on; rejected on the host
+    d = torch.zeros(16, device="cuda")
+    i = torch.zeros(16, dtype=torch.int32, device="cuda")
+    w = B.make_weights(d, None, torch.zeros(shape.stride, dtype=torch.uint8, device="cuda"),
+                       torch.zeros(shape.stride, dtype=torch.uint8, device="cuda"), shape.stride)
+    assert B.coli_moe_forward_noalloc(dims, w, d, 57, d, i, i, i, i, None, d) == B.COLI_ENOMEM
