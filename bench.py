@@ -198,6 +198,8 @@ def run_ours(args, rank, world, local_rank):
     y_host = torch.empty(T, H, dtype=torch.float32).pin_memory()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    flush_read = torch.zeros(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     # union size of every batch in the pool (deterministic), for the byte counts
@@ -211,42 +213,64 @@ def run_ours(args, rank, world, local_rank):
     def step(i, ev=None):
         x = xs[i % R]
         if ev:
-            ev[0].record(stream)
+            ev[0].record()
         B.check(B.coli_moe_route_union(dims, wr, bias, x, T, bufs.idx, bufs.w, None,
                                        bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
                                        bufs.ws), "route_union")
         if ev:
-            ev[1].record(stream)
+            ev[1].record()
         B.check(B.coli_moe_gate_up(dims, weights, x, T, bufs.union_ids, bufs.n_union,
                                    bufs.offsets, bufs.assign, bufs.ws), "gate_up")
         if ev:
-            ev[2].record(stream)
+            ev[2].record()
         B.check(B.coli_moe_down(dims, weights, T, bufs.w, bufs.union_ids, bufs.n_union,
                                 bufs.offsets, bufs.assign, None, bufs.y, bufs.ws), "down")
         if ev:
-            ev[3].record(stream)
+            ev[3].record()
 
     def flush():
+        # write 2x L2, then read another 2x L2: our data is evicted and L2 is left holding
+        # clean lines, so no write-back of the flush lands inside the timed interval
         flush_buf.zero_()
+        torch.sum(flush_read, dim=0, keepdim=True, out=flush_sink)
+
+    # The timed steps run as CUDA graphs (flush + 3 launches per step, with event-record
+    # nodes around each launch), so the GPU never waits for the host to enqueue work.
+    def capture(first, n):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+               for _ in range(n)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                flush()
+                step(first + i, evs[i])
+        return g, evs
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id)
     sampler.start()
     time.sleep(0.2)
-    for i in range(args.warmup):
-        flush()
-        step(i)
+    K = args.steps
+    G = min(K, 128)
+    chunks = [(c, min(G, K - c)) for c in range(0, K, G)]
+    graphs = {}
+    for (c, n) in chunks:
+        if n not in graphs:
+            graphs[n] = capture(args.warmup, n)
+    if args.warmup:
+        gw, _ = capture(0, args.warmup)
+        gw.replay()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    seg_rows = []
     t0 = time.time()
-    for i in range(K):
-        flush()
-        step(args.warmup + i, evs[i])
-    torch.cuda.synchronize(dev)
+    for (c, n) in chunks:
+        g, evs = graphs[n]
+        g.replay()
+        torch.cuda.synchronize(dev)
+        seg_rows += [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(n)]
     t1 = time.time()
     if world > 1:
         torch.distributed.barrier()
@@ -254,8 +278,9 @@ def run_ours(args, rank, world, local_rank):
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
+    del graphs
 
-    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(K)])
+    seg = np.array(seg_rows)
     step_ms = seg.sum(axis=1)
     total_ms = float(step_ms.sum())
     st, bits = B.coli_moe_read_status(bufs.ws)
@@ -299,7 +324,8 @@ def run_ours(args, rank, world, local_rank):
     blob = s.blob_bytes
     gu_bytes_expert = 2 * (I * H // 2) + 2 * (I * H // 64) * 2
     dn_bytes_expert = H * I // 2 + H * (I // 64) * 2
-    nu = np.array([n_union[(args.warmup + i) % R] for i in range(K)], dtype=np.float64)
+    nu = np.array([n_union[(args.warmup + i) % R] for (c, n) in chunks for i in range(n)],
+                  dtype=np.float64)
     units = nu + s.n_shared
     x_bytes = T * H * 4
     h_bytes = (T * k + T * s.n_shared) * I * 4
@@ -342,7 +368,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "tokens_per_step": T, "hidden": H, "intermediate": I,
                    "experts": E, "top_k": k, "shared_experts": s.n_shared,
                    "weights": "gs64 int4, fp16 scales", "activations": "fp32",
-                   "l2": "flushed (2x L2 write) before every step, outside the timed intervals",
+                   "l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
+                   "timing": "CUDA graphs of up to 128 steps; events around each launch",
                    "token_pool": R, "parallelism": f"replicas x{world}",
                    "mean_union": float(nu.mean())},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gb_s"],

@@ -137,7 +137,7 @@ GemvParams gemv_params(const coli_moe_dims* d, const coli_moe_weights* wt, const
     p.offsets = offsets;
     p.assign = assign;
     p.wts = w;
-    p.h = reinterpret_cast<float*>((uint8_t*)ws + ws_layout(d, T).h);
+    p.hd = (uint8_t*)ws + ws_layout(d, T).h;
     p.y = y;
     p.residual = residual;
     p.status = &reinterpret_cast<WsHeader*>(ws)->status;

@@ -33,31 +33,121 @@
 namespace coli {
 namespace {
 
-constexpr int kV = 8;            // values per consumer thread and stage
 constexpr int kBarFull = 0;      // mbarrier slots in shared memory
 constexpr int kMaxStages = 16;
+constexpr int kMaxChunks = 64;      // pending chunks per flush
 
-// 8 int4 values of one 32-bit word -> 4 exact float pairs (columns (0,1) (2,3) (4,5) (6,7)).
-// Nibble k sits at bits 4k.  For k <= 4 the nibble lies inside a float mantissa whose
-// exponent gives bit 4k the weight 1: (w & 0xF<<4k) ^ (exp_k | 8<<4k) has the value
-// 2^(23-4k) + (n ^ 8), and n ^ 8 = q + 8 for the two's-complement nibble n of q.
-// Nibbles 5..7 are taken from w >> 12 (positions of nibbles 2..4).  Subtracting
-// 2^(23-4k) + 8 is exact, so the pairs hold q exactly.
-__device__ __forceinline__ void dequant8(uint32_t w, uint64_t (&q)[4])
+// dp4a: c + sum_i a_i * b_i over the four bytes, exact in 32-bit integers; a's bytes
+// unsigned, b's bytes signed (dp4a_us) or unsigned (dp4a_uu, wrapping mod 2^32)
+__device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c)
 {
-    const uint32_t w2 = w >> 12;
-    const uint32_t f0 = and_xor(w, 0x0000000Fu, 0x4B000008u);   // 2^23 + q + 8
-    const uint32_t f1 = and_xor(w, 0x000000F0u, 0x49000080u);   // 2^19 + q + 8
-    const uint32_t f2 = and_xor(w, 0x00000F00u, 0x47000800u);   // 2^15 + q + 8
-    const uint32_t f3 = and_xor(w, 0x0000F000u, 0x45008000u);   // 2^11 + q + 8
-    const uint32_t f4 = and_xor(w, 0x000F0000u, 0x43080000u);   // 2^7  + q + 8
-    const uint32_t f5 = and_xor(w2, 0x00000F00u, 0x47000800u);
-    const uint32_t f6 = and_xor(w2, 0x0000F000u, 0x45008000u);
-    const uint32_t f7 = and_xor(w2, 0x000F0000u, 0x43080000u);
-    q[0] = fadd2(pk2(f0, f1), pk2f(-8388616.0f, -524296.0f));
-    q[1] = fadd2(pk2(f2, f3), pk2f(-32776.0f, -2056.0f));
-    q[2] = fadd2(pk2(f4, f5), pk2f(-136.0f, -32776.0f));
-    q[3] = fadd2(pk2(f6, f7), pk2f(-2056.0f, -136.0f));
+    int32_t d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c)
+{
+    uint32_t d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"((uint32_t)c));
+    return (int32_t)d;
+}
+
+// Activations of one 32-column unit as 8-bit digits.  With m = max |x_c| over the unit,
+// X_c = clamp(x_c * 126 / m, -126, 126) is written as
+//     X_c = a_c + b_c / 256 + c_c / 65536 + r_c,  a_c in [-126, 126] (signed),
+//     b_c, c_c in [0, 255] (unsigned),  0 <= r_c < 2^-16
+// (floor digits, the last one rounded), so that
+//     sum_c q_c x_c = (m / (126 * 65536)) * sum_c q_c (65536 a_c + 256 b_c + c_c)
+// up to about 1.2e-7 m per column, with the integer sum exact in int32 (below 2^31 for
+// |q| <= 8 over 32 columns).  Weight nibbles arrive in offset binary n' = q + 8, so each
+// digit's dp4a chain starts at -8 * sum_c digit_c.  Digits are packed in the byte order
+// of the nibble words: word wi holds columns 8wi + {0,2,4,6} (low nibbles, even slot) and
+// 8wi + {1,3,5,7} (high nibbles, odd slot).
+__device__ __forceinline__ void load_digits(const float* src, uint32_t (&dg)[3][8],
+                                            int32_t (&corr)[3], float& fac)
+{
+    float xv[32];
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int q4 = 0; q4 < 8; q4++) {
+        const float4 v = s4[q4];
+        xv[4 * q4] = v.x;
+        xv[4 * q4 + 1] = v.y;
+        xv[4 * q4 + 2] = v.z;
+        xv[4 * q4 + 3] = v.w;
+    }
+    float mx = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 32; c++) mx = fmaxf(mx, fabsf(xv[c]));
+    const float inv = mx > 0.0f ? 126.0f / mx : 0.0f;
+    fac = mx * (1.0f / (126.0f * 65536.0f));
+#pragma unroll
+    for (int d = 0; d < 3; d++) {
+        corr[d] = 0;
+#pragma unroll
+        for (int q = 0; q < 8; q++) dg[d][q] = 0u;
+    }
+#pragma unroll
+    for (int c = 0; c < 32; c++) {
+        const float X = fminf(fmaxf(xv[c] * inv, -126.0f), 126.0f);
+        const float a = floorf(X);
+        const float r1 = (X - a) * 256.0f;
+        const float bq = floorf(r1);
+        const float cq = fminf(rintf((r1 - bq) * 256.0f), 255.0f);
+        const int di[3] = {(int)a, (int)bq, (int)cq};
+        const int wi = c >> 3, k = c & 7;
+        const int slot = 2 * wi + (k & 1), byte = k >> 1;
+#pragma unroll
+        for (int d = 0; d < 3; d++) {
+            dg[d][slot] |= ((uint32_t)di[d] & 0xFFu) << (8 * byte);
+            corr[d] -= 8 * di[d];
+        }
+    }
+}
+
+// A warp turns 32 consecutive activations (lane l holds column l) into one digit record
+// with the same digits as load_digits: words 0..23 are the packed planes (plane d, slot
+// 2wi + p holds columns 8wi + 2b + p at byte b), words 24..26 the corrections
+// -8 * sum(digit), word 27 the factor m / (126 * 65536).
+__device__ __forceinline__ void store_digit_record(float hv, int lane, uint32_t* rec)
+{
+    float mx = fabsf(hv);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.0f ? 126.0f / mx : 0.0f;
+    const float X = fminf(fmaxf(hv * inv, -126.0f), 126.0f);
+    const float a = floorf(X);
+    const float r1 = (X - a) * 256.0f;
+    const float bq = floorf(r1);
+    const float cq = fminf(rintf((r1 - bq) * 256.0f), 255.0f);
+    const int di[3] = {(int)a, (int)bq, (int)cq};
+    // lane L < 24 assembles word L: plane d = L / 8, slot s = L % 8
+    const int d_me = lane >> 3, slot = lane & 7, wi = slot >> 1, par = slot & 1;
+    uint32_t word = 0;
+#pragma unroll
+    for (int d = 0; d < 3; d++) {
+#pragma unroll
+        for (int bb = 0; bb < 4; bb++) {
+            const int src = 8 * wi + 2 * bb + par;
+            const int v = __shfl_sync(0xffffffffu, di[d], src);
+            if (d == d_me) word |= ((uint32_t)v & 0xFFu) << (8 * bb);
+        }
+    }
+    int sums[3];
+#pragma unroll
+    for (int d = 0; d < 3; d++) {
+        int sv = di[d];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
+        sums[d] = sv;
+    }
+    uint32_t out = word;
+    if (lane == 24) out = (uint32_t)(-8 * sums[0]);
+    if (lane == 25) out = (uint32_t)(-8 * sums[1]);
+    if (lane == 26) out = (uint32_t)(-8 * sums[2]);
+    if (lane == 27) out = __float_as_uint(mx * (1.0f / (126.0f * 65536.0f)));
+    if (lane < kDigitRecWords) rec[lane] = out;
 }
 
 // Transposing butterfly over W*2 lanes: at each level the lane with bit W set keeps the
@@ -112,7 +202,8 @@ __device__ __forceinline__ Seg seg_info(const GemvParams& p, int s)
     return g;
 }
 
-// token id and routing weight of token mm of a segment
+// token id and routing weight of token mm of a segment (the gate/up launch has no
+// routing weights: p.wts is null there and wt is 0)
 __device__ __forceinline__ void seg_token(const GemvParams& p, const Seg& g, int mm, int& tok,
                                           float& wt)
 {
@@ -122,19 +213,26 @@ __device__ __forceinline__ void seg_token(const GemvParams& p, const Seg& g, int
     } else {
         const int a = p.assign[g.base + mm];
         tok = a / p.k;
-        wt = p.wts[a];
+        wt = p.wts ? p.wts[a] : 0.0f;
     }
 }
 
 template <int MODE>
 __device__ __forceinline__ void cta_rows(const GemvParams& p, int nseg, int64_t& r0, int64_t& r1)
 {
-    const int64_t R = (MODE == 0) ? (int64_t)nseg * p.N : (int64_t)p.N;
-    r0 = R * blockIdx.x / gridDim.x;
-    r1 = R * (blockIdx.x + 1) / gridDim.x;
+    if (MODE == 0) {
+        // whole 32-row units, so every unit of h is finished by one CTA
+        const int64_t R = (int64_t)nseg * (p.N / 32);
+        r0 = 32 * (R * blockIdx.x / gridDim.x);
+        r1 = 32 * (R * (blockIdx.x + 1) / gridDim.x);
+    } else {
+        r0 = (int64_t)p.N * blockIdx.x / gridDim.x;
+        r1 = (int64_t)p.N * (blockIdx.x + 1) / gridDim.x;
+    }
 }
 
-// Calls f(seg, row0, nrows) for the CTA's pieces in the fixed order.
+// Calls f(seg, row0, nrows) for the CTA's pieces in the fixed order.  A piece is a run of
+// rows of one segment, at most p.PR rows long (the partial-sum buffer holds one piece).
 template <int MODE, class F>
 __device__ __forceinline__ void for_each_piece(const GemvParams& p, int nseg, F&& f)
 {
@@ -145,20 +243,36 @@ __device__ __forceinline__ void for_each_piece(const GemvParams& p, int nseg, F&
         while (r < r1) {
             const int s = (int)(r / p.N);
             const int64_t end = min(r1, (int64_t)(s + 1) * p.N);
-            f(s, (int)(r - (int64_t)s * p.N), (int)(end - r));
+            for (int64_t q = r; q < end; q += p.PR)
+                f(s, (int)(q - (int64_t)s * p.N), (int)min((int64_t)p.PR, end - q));
             r = end;
         }
     } else {
         if (r1 > r0)
-            for (int s = 0; s < nseg; s++) f(s, (int)r0, (int)(r1 - r0));
+            for (int s = 0; s < nseg; s++)
+                for (int64_t q = r0; q < r1; q += p.PR)
+                    f(s, (int)q, (int)min((int64_t)p.PR, r1 - q));
     }
 }
 
+// Bookkeeping of a chunk (piece x up to MAXM tokens) whose partial sums wait in shared
+// memory for the CTA's next flush.
+struct ChunkMeta {   // 60 bytes
+    int base, c0, M, row0, nrows, part_off, u;
+    int tok[4];
+    float wt[4];
+};
+
+// Consumer threads per CTA and values per thread per stage, by tokens per chunk.
+__host__ __device__ constexpr int consumers_for(int maxm) { return maxm == 4 ? 192 : 384; }
+__host__ __device__ constexpr int values_for(int maxm) { return 8; }
+
 template <int MODE, int MAXM, int L>
-__global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
+__global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     gemv_kernel(const __grid_constant__ GemvParams p)
 {
-    constexpr int NCONS = (MAXM == 4) ? 192 : 384;
+    constexpr int NCONS = consumers_for(MAXM);
+    constexpr int kV = values_for(MAXM);
     constexpr int NMAT = (MODE == 0) ? 2 : 1;
     constexpr int RPT = kV / (MAXM * NMAT);
     static_assert(RPT >= 1 && RPT * MAXM * NMAT == kV, "value layout");
@@ -213,7 +327,8 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
                     if (!dead) {
                         uint8_t* dst = vec + b * p.vec_bytes;
                         const uint32_t rowb = (uint32_t)K * 4u;
-                        mbar_arrive_expect_tx(&vfull[b], rowb * M);
+                        mbar_arrive_expect_tx(&vfull[b], MODE == 0 ? rowb * M
+                                                                   : (uint32_t)(p.U * kDigitRecBytes) * M);
                         if (MODE == 0) {
                             for (int m = 0; m < M; m++) {
                                 int tok;
@@ -222,7 +337,8 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
                                 bulk_g2s(dst + m * rowb, p.x + (size_t)tok * p.H, rowb, &vfull[b]);
                             }
                         } else {
-                            bulk_g2s(dst, p.h + (size_t)(g.base + c0) * p.I, rowb * M, &vfull[b]);
+                            bulk_g2s(dst, p.hd + (size_t)(g.base + c0) * p.U * kDigitRecBytes,
+                                     (uint32_t)(p.U * kDigitRecBytes) * M, &vfull[b]);
                         }
                     }
                     vit++;
@@ -280,11 +396,15 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
     const int wg = (U >= 32) ? (j >> 5) : 0;
     const int lane_l = lane & (L - 1);
     bool dead = false;
+    float* part = red;                                   // partial sums of pending chunks
+    ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + p.off_meta);
+    int nch = 0;                                         // pending chunks (CTA-uniform)
+    uint32_t part_used = 0;
+    int64_t r0, r1;
+    cta_rows<MODE>(p, nseg, r0, r1);
 
     if (MODE == 1) {
         // this CTA owns rows [r0, r1) of y for every token: start from residual or zero
-        int64_t r0, r1;
-        cta_rows<MODE>(p, nseg, r0, r1);
         const int nrw = (int)(r1 - r0);
         for (int f = tid; f < p.T * nrw; f += NCONS) {
             const int t = f / nrw, r = (int)r0 + (f - t * nrw);
@@ -292,17 +412,96 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
         }
     }
     if (p.resident) {
-        if (!mbar_wait(&vfull[0], 0, p.status, 21)) dead = true;
+        if (!dead && !mbar_wait(&vfull[0], 0, p.status, 21)) dead = true;
     }
 
-    uint64_t xr[MAXM][16];   // activation pairs of this thread's column unit
+    // Sum the pending chunks' partials: SwiGLU into h (mode 0) or the fixed-order combine
+    // into y (mode 1: one thread per output row walks the chunks in order).
+    auto flush = [&]() {
+        named_bar(1, NCONS);
+        if (MODE == 0) {
+            // one warp per (chunk, token, 32-row unit): lane l finishes h of row 32u + l,
+            // then the warp writes the unit as a digit record for the down projection
+            const int nwarps = NCONS / 32;
+            for (int c = 0; c < nch; c++) {
+                const ChunkMeta& cm = meta[c];
+                const float* pc = part + cm.part_off;
+                const int units = cm.nrows / 32;
+                for (int task = warp; task < units * cm.M; task += nwarps) {
+                    const int m = task / units, uu = task - m * units;
+                    const int rl_ = uu * 32 + lane;
+                    const float* q = pc + ((size_t)(rl_ * MAXM + m) * NMAT) * nwg;
+                    float gs = 0.0f, us = 0.0f;
+                    for (int w2 = 0; w2 < nwg; w2++) {
+                        gs += q[w2];
+                        us += q[nwg + w2];
+                    }
+                    const float hv = gs / (1.0f + expf(-gs)) * us;
+                    const int urow = (cm.row0 >> 5) + uu;   // unit index along I
+                    uint32_t* rec = reinterpret_cast<uint32_t*>(
+                        p.hd + ((size_t)(cm.base + cm.c0 + m) * (p.I / 32) + urow) * kDigitRecBytes);
+                    store_digit_record(hv, lane, rec);
+                }
+            }
+        } else {
+            const int nrw = (int)(r1 - r0);
+            for (int rr = tid; rr < nrw; rr += NCONS) {
+                const int r = (int)r0 + rr;
+                for (int c = 0; c < nch; c++) {
+                    const ChunkMeta& cm = meta[c];
+                    const int rl_ = r - cm.row0;
+                    if (rl_ < 0 || rl_ >= cm.nrows) continue;
+                    const float* pc = part + cm.part_off;
+                    for (int m = 0; m < cm.M; m++) {
+                        const float* q = pc + (size_t)(rl_ * MAXM + m) * nwg;
+                        float d = 0.0f;
+                        for (int w2 = 0; w2 < nwg; w2++) d += q[w2];
+                        float* yp = p.y + (size_t)cm.tok[m] * p.H + r;
+                        *yp = *yp + cm.wt[m] * d;
+                    }
+                }
+            }
+        }
+        named_bar(1, NCONS);
+        nch = 0;
+        part_used = 0;
+    };
+
+    // activations of this thread's 32-column unit as three int8 digits per column,
+    // packed in the byte order of the offset-binary nibble words (see load_digits)
+    uint32_t dg[MAXM][3][8];
+    int32_t dcorr[MAXM][3];
+    float dfac[MAXM];
     uint32_t it = 0, vit = 0;
 
     for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
         const Seg g = seg_info(p, s);
         for (int c0 = 0; c0 < g.count; c0 += MAXM) {
             const int M = min(MAXM, g.count - c0);
-            // ---- activations for this chunk into registers
+            const uint32_t need = (uint32_t)nrows * MAXM * NMAT * nwg;
+            if (nch == kMaxChunks || part_used + need > p.part_cap) flush();
+            const uint32_t off = part_used;
+            if (tid == 0) {
+                ChunkMeta& cm = meta[nch];
+                cm.base = g.base;
+                cm.c0 = c0;
+                cm.M = M;
+                cm.row0 = row0;
+                cm.nrows = nrows;
+                cm.part_off = (int)off;
+                cm.u = g.u;
+                for (int m = 0; m < 4; m++) {
+                    int tok = 0;
+                    float wt = 0.0f;
+                    if (m < M) seg_token(p, g, c0 + m, tok, wt);
+                    cm.tok[m] = tok;
+                    cm.wt[m] = wt;
+                }
+            }
+            nch++;
+            part_used += need;
+            float* pc = part + off;
+            // ---- activations for this chunk into registers (as int8 digits)
             const float* vsrc;
             int b = 0;
             if (!p.resident) {
@@ -322,17 +521,32 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
                         seg_token(p, g, c0 + m, tok, wt);
                         row_in_vec = tok;
                     }
-                    const float4* src =
-                        reinterpret_cast<const float4*>(vsrc + (size_t)row_in_vec * K + 32 * j);
+                    if (MODE == 0) {
+                        load_digits(vsrc + (size_t)row_in_vec * K + 32 * j, dg[m], dcorr[m], dfac[m]);
+                    } else {
+                        const uint4* rec = reinterpret_cast<const uint4*>(
+                            reinterpret_cast<const uint8_t*>(vsrc) +
+                            ((size_t)m * p.U + j) * kDigitRecBytes);
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; q4++) {
-                        const float4 v4 = src[q4];
-                        xr[m][2 * q4] = pk2f(v4.x, v4.y);
-                        xr[m][2 * q4 + 1] = pk2f(v4.z, v4.w);
+                        for (int d = 0; d < 3; d++) {
+                            const uint4 r0v = rec[2 * d], r1v = rec[2 * d + 1];
+                            dg[m][d][0] = r0v.x; dg[m][d][1] = r0v.y; dg[m][d][2] = r0v.z; dg[m][d][3] = r0v.w;
+                            dg[m][d][4] = r1v.x; dg[m][d][5] = r1v.y; dg[m][d][6] = r1v.z; dg[m][d][7] = r1v.w;
+                        }
+                        const uint4 tail = rec[6];
+                        dcorr[m][0] = (int32_t)tail.x;
+                        dcorr[m][1] = (int32_t)tail.y;
+                        dcorr[m][2] = (int32_t)tail.z;
+                        dfac[m] = __uint_as_float(tail.w);
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 16; q++) xr[m][q] = 0ull;
+                    for (int d = 0; d < 3; d++) {
+                        dcorr[m][d] = 0;
+#pragma unroll
+                        for (int q = 0; q < 8; q++) dg[m][d][q] = 0u;
+                    }
+                    dfac[m] = 0.0f;
                 }
             }
             if (!p.resident) {
@@ -353,38 +567,55 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
 #pragma unroll
                 for (int q = 0; q < kV; q++) v[q] = 0.0f;
                 if (active) {
+                    // every row slot of the stage is computed (slots past nr read stale but
+                    // in-bounds shared memory and are discarded below), so the loads of all
+                    // rows issue together and the dp4a chains of different rows interleave
+                    uint4 wv[RPT][NMAT];
+                    float scv[RPT][NMAT];
 #pragma unroll
                     for (int i = 0; i < RPT; i++) {
                         const int rr = rho + p.rl * i;
-                        if (rr < nr) {
 #pragma unroll
-                            for (int mt = 0; mt < NMAT; mt++) {
-                                const uint4 wv = *reinterpret_cast<const uint4*>(
-                                    sbase + (size_t)mt * p.SR * (K / 2) + (size_t)rr * (K / 2) + 16 * j);
-                                const float sc = __half2float(*reinterpret_cast<const __half*>(
-                                    sbase + p.stage_sc_off + mt * p.sc_area + delta + rr * (K / 32) +
-                                    (j >> 1) * 2));
-                                uint64_t acc[MAXM];
+                        for (int mt = 0; mt < NMAT; mt++) {
+                            wv[i][mt] = *reinterpret_cast<const uint4*>(
+                                sbase + (size_t)mt * p.SR * (K / 2) + (size_t)rr * (K / 2) + 16 * j);
+                            scv[i][mt] = __half2float(*reinterpret_cast<const __half*>(
+                                sbase + p.stage_sc_off + mt * p.sc_area + delta + rr * (K / 32) +
+                                (j >> 1) * 2));
+                        }
+                    }
 #pragma unroll
-                                for (int m = 0; m < MAXM; m++) acc[m] = 0ull;
-                                const uint32_t wds[4] = {wv.x, wv.y, wv.z, wv.w};
+                    for (int i = 0; i < RPT; i++) {
 #pragma unroll
-                                for (int wi = 0; wi < 4; wi++) {
-                                    uint64_t qq[4];
-                                    dequant8(wds[wi], qq);
+                        for (int mt = 0; mt < NMAT; mt++) {
+                            // offset-binary nibbles n' = q + 8 as bytes: even columns of word wi
+                            // in lo[wi], odd columns in hi[wi]
+                            const uint32_t wds[4] = {wv[i][mt].x, wv[i][mt].y, wv[i][mt].z, wv[i][mt].w};
+                            uint32_t lo[4], hi[4];
 #pragma unroll
-                                    for (int m = 0; m < MAXM; m++) {
-                                        if (m < M) {
+                            for (int wi = 0; wi < 4; wi++) {
+                                lo[wi] = and_xor(wds[wi], 0x0F0F0F0Fu, 0x08080808u);
+                                hi[wi] = and_xor(wds[wi] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+                            }
 #pragma unroll
-                                            for (int pi = 0; pi < 4; pi++)
-                                                acc[m] = ffma2(qq[pi], xr[m][wi * 4 + pi], acc[m]);
-                                        }
+                            for (int m = 0; m < MAXM; m++) {
+                                if (m < M) {
+                                    // two independent chains per digit (even / odd columns)
+                                    int32_t e0 = dcorr[m][0], o0 = 0;
+                                    int32_t e1 = dcorr[m][1], o1 = 0;
+                                    int32_t e2 = dcorr[m][2], o2 = 0;
+#pragma unroll
+                                    for (int wi = 0; wi < 4; wi++) {
+                                        e0 = dp4a_us(lo[wi], dg[m][0][2 * wi], e0);
+                                        o0 = dp4a_us(hi[wi], dg[m][0][2 * wi + 1], o0);
+                                        e1 = dp4a_uu(lo[wi], dg[m][1][2 * wi], e1);
+                                        o1 = dp4a_uu(hi[wi], dg[m][1][2 * wi + 1], o1);
+                                        e2 = dp4a_uu(lo[wi], dg[m][2][2 * wi], e2);
+                                        o2 = dp4a_uu(hi[wi], dg[m][2][2 * wi + 1], o2);
                                     }
-                                }
-#pragma unroll
-                                for (int m = 0; m < MAXM; m++) {
-                                    const float2 a = unpk2(acc[m]);
-                                    v[(i * MAXM + m) * NMAT + mt] = sc * (a.x + a.y);
+                                    // sum_c q_c * (65536 a_c + 256 b_c + c_c), exact in int32
+                                    const int32_t S = ((e0 + o0) * 256 + (e1 + o1)) * 256 + (e2 + o2);
+                                    v[(i * MAXM + m) * NMAT + mt] = (float)S * (dfac[m] * scv[i][mt]);
                                 }
                             }
                         }
@@ -393,59 +624,50 @@ __global__ void __launch_bounds__((MAXM == 4 ? 192 : 384) + 32, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
 
-                float* rbuf = red + (size_t)(it & 1) * p.rl * nwg * kV;
                 if (active) {
                     Bfly<kV, L / 2>::run(v, lane);
+                    // value index vi = (i*MAXM + m)*NMAT + mt  ->  row r + rho + rl*i
                     if (kV >= L) {
 #pragma unroll
-                        for (int i2 = 0; i2 < kV / L; i2++)
-                            rbuf[((size_t)rho * nwg + wg) * kV + i2 + (kV / L) * lane_l] = v[i2];
+                        for (int i2 = 0; i2 < kV / L; i2++) {
+                            const int vi = i2 + (kV / L) * lane_l;
+                            const int i = vi / (MAXM * NMAT), mm = vi % (MAXM * NMAT);
+                            const int rr = rho + p.rl * i;
+                            if (rr < nr)
+                                pc[((size_t)(r + rr) * MAXM * NMAT + mm) * nwg + wg] = v[i2];
+                        }
                     } else {
                         constexpr int REP = (kV >= L) ? 1 : L / kV;
-                        if ((lane_l % REP) == 0) rbuf[((size_t)rho * nwg + wg) * kV + lane_l / REP] = v[0];
-                    }
-                }
-                named_bar(1, NCONS);
-                // ---- finalize: one thread per (row, token)
-                for (int f = tid; f < p.SR * M; f += NCONS) {
-                    const int m = f / p.SR;
-                    const int rr = f - m * p.SR;
-                    if (rr >= nr) continue;
-                    const int rho2 = rr % p.rl, i = rr / p.rl;
-                    const float* rv = rbuf + (size_t)rho2 * nwg * kV;
-                    if (MODE == 0) {
-                        float gs = 0.0f, us = 0.0f;
-                        for (int w2 = 0; w2 < nwg; w2++) {
-                            gs += rv[w2 * kV + (i * MAXM + m) * 2 + 0];
-                            us += rv[w2 * kV + (i * MAXM + m) * 2 + 1];
+                        if ((lane_l % REP) == 0) {
+                            const int vi = lane_l / REP;
+                            const int i = vi / (MAXM * NMAT), mm = vi % (MAXM * NMAT);
+                            const int rr = rho + p.rl * i;
+                            if (rr < nr)
+                                pc[((size_t)(r + rr) * MAXM * NMAT + mm) * nwg + wg] = v[0];
                         }
-                        const float hv = gs / (1.0f + expf(-gs)) * us;
-                        p.h[(size_t)(g.base + c0 + m) * p.I + row + rr] = hv;
-                    } else {
-                        float d = 0.0f;
-                        for (int w2 = 0; w2 < nwg; w2++) d += rv[w2 * kV + i * MAXM + m];
-                        int tok;
-                        float wt;
-                        seg_token(p, g, c0 + m, tok, wt);
-                        float* yp = p.y + (size_t)tok * p.H + row + rr;
-                        *yp = *yp + wt * d;
                     }
                 }
                 it++;
             }
         }
     });
+    flush();
 }
 
 template <int MODE, int MAXM, int L>
 cudaError_t launch_one(const GemvParams& p, const GemvConfig& c, cudaStream_t s)
 {
     auto kern = gemv_kernel<MODE, MAXM, L>;
-    static bool attr_set = false;   // per instantiation; the attribute is per device
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)c.smem);
+    // the opt-in shared-memory size is set once per device and size (host-side cache)
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    (void)attr_set;
+    if (dev < 0 || dev >= 64 || set_bytes[dev] < (int)c.smem) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)c.smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) set_bytes[dev] = (int)c.smem;
+    }
     kern<<<c.grid, c.consumers + 32, c.smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -489,7 +711,8 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
         c.maxm = p.T <= 1 ? 1 : (p.T <= 2 ? 2 : (p.T <= 4 ? 4 : 2));
     else
         c.maxm = p.T <= 1 ? 1 : (p.T <= 2 ? 2 : 4);
-    c.consumers = c.maxm == 4 ? 192 : 384;
+    c.consumers = consumers_for(c.maxm);
+    const int kV = values_for(c.maxm);
     if (p.U >= 32) {
         if (p.U % 32 || p.U > c.consumers) return false;
         c.lanes = 32;
@@ -501,11 +724,20 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
     c.rpt = kV / (c.maxm * NMAT);
     p.SR = p.rl * c.rpt;
     const int nwg = p.U >= 32 ? p.U / 32 : 1;
-    const uint32_t red_bytes = 2u * p.rl * nwg * kV * 4u;
-    p.off_red = 512;
+    // partial sums: a decode CTA's whole share of rows fits, larger shares flush in pieces
+    p.part_cap = 4096;                                    // 16 KB
+    const uint32_t per_row = (uint32_t)c.maxm * NMAT * nwg;
+    p.PR = (int)(p.part_cap / per_row);
+    if (mode == 0) p.PR = p.PR / 32 * 32;   // pieces are whole 32-row units
+    if (p.PR < 1) return false;
+    p.off_meta = 512;
+    p.off_red = align_up(p.off_meta + 64u * 64u, 128);    // kMaxChunks x sizeof(ChunkMeta) <= 64
+    const uint32_t red_bytes = p.part_cap * 4u;
     const uint64_t xres = (uint64_t)p.T * p.H * 4ull;
     p.resident = (mode == 0 && xres <= 100u * 1024u) ? 1 : 0;
-    p.vec_bytes = p.resident ? (uint32_t)xres : (uint32_t)c.maxm * p.K * 4u;
+    p.vec_bytes = p.resident ? (uint32_t)xres
+                             : (mode == 0 ? (uint32_t)c.maxm * p.K * 4u
+                                          : (uint32_t)c.maxm * p.U * kDigitRecBytes);
     const uint32_t nvec = p.resident ? 1 : 2;
     p.off_vec = align_up(p.off_red + red_bytes, 128);
     p.off_stage = align_up(p.off_vec + nvec * p.vec_bytes, 128);

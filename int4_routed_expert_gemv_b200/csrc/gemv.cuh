@@ -18,6 +18,9 @@ struct GemvParams {
     int SR;         // rows per pipeline stage = rl * RPT
     int NS;         // pipeline stages
     int resident;   // gate/up: the whole batch's x lives in shared memory
+    int PR;         // max rows of one piece (one chunk's partials fit the buffer)
+    uint32_t part_cap;  // floats in the partial-sum buffer
+    uint32_t off_meta;  // chunk bookkeeping
     // shared-memory layout (bytes)
     uint32_t off_red, off_vec, off_stage;
     uint32_t vec_bytes;     // one vector buffer
@@ -36,11 +39,18 @@ struct GemvParams {
     const int32_t* offsets;   // [E+1]
     const int32_t* assign;    // [T*k]
     const float* wts;         // [T][k] routing weights
-    float* h;                 // [T*k + T][I] SwiGLU activations (workspace)
+    uint8_t* hd;              // SwiGLU activations h as digit records (workspace):
+                              // row p (assign position, or T*k + t for the shared
+                              // expert) holds I/32 records of kDigitRecBytes
     float* y;                 // [T][H] output
     const float* residual;    // [T][H] or null (down: y = residual + MoE)
     uint32_t* status;         // workspace header
 };
+
+// One 32-column unit of activations in digit form: three planes of 8 packed bytes, the
+// three dp4a corrections and the scale factor (28 words).
+constexpr int kDigitRecWords = 28;
+constexpr int kDigitRecBytes = kDigitRecWords * 4;
 
 struct GemvConfig {
     int maxm;         // tokens per chunk (register-resident activations)

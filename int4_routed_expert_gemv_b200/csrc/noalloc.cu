@@ -119,7 +119,7 @@ extern "C" coli_status coli_moe_forward_noalloc(const coli_moe_dims* d, const co
         p.offsets = offsets;
         p.assign = assign;
         p.wts = w;
-        p.h = reinterpret_cast<float*>(base + kHeaderBytes);
+        p.hd = base + kHeaderBytes;
         p.y = mode == 1 ? y : nullptr;
         p.residual = mode == 1 ? residual : nullptr;
         p.status = reinterpret_cast<uint32_t*>(base);

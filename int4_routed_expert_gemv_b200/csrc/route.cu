@@ -111,25 +111,39 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     for (int r = 0; r < RB; r++)
 #pragma unroll
         for (int t = 0; t < kSmallT; t++) acc[r][t] = 0.0;
-    for (int c4 = tid; c4 < H4; c4 += 256) {
-        float4 wv[RB];
+    // all of this thread's router loads are issued before any arithmetic, so the CTA
+    // waits for one memory round trip per pass (one pass up to H = 8192)
+    constexpr int MAXIT = 8;
+    for (int base = 0; base < H4; base += 256 * MAXIT) {
+        float4 wv[RB][MAXIT];
 #pragma unroll
-        for (int r = 0; r < RB; r++)
-            wv[r] = (e0 + r < p.E) ? __ldcs(reinterpret_cast<const float4*>(p.w_router) +
-                                            (size_t)(e0 + r) * H4 + c4)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int it = 0; it < MAXIT; it++) {
+            const int c4 = base + it * 256 + tid;
 #pragma unroll
-        for (int t = 0; t < kSmallT; t++) {
-            if (t < p.T) {
-                const float4 xv = load_x4<XT>(x, (size_t)t * H4 + c4);
+            for (int r = 0; r < RB; r++)
+                wv[r][it] = (c4 < H4 && e0 + r < p.E)
+                                ? __ldcs(reinterpret_cast<const float4*>(p.w_router) +
+                                         (size_t)(e0 + r) * H4 + c4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-                for (int r = 0; r < RB; r++) {
-                    double a = acc[r][t];
-                    a = fma((double)xv.x, (double)wv[r].x, a);
-                    a = fma((double)xv.y, (double)wv[r].y, a);
-                    a = fma((double)xv.z, (double)wv[r].z, a);
-                    a = fma((double)xv.w, (double)wv[r].w, a);
-                    acc[r][t] = a;
+        for (int it = 0; it < MAXIT; it++) {
+            const int c4 = base + it * 256 + tid;
+            if (c4 < H4) {
+#pragma unroll
+                for (int t = 0; t < kSmallT; t++) {
+                    if (t < p.T) {
+                        const float4 xv = load_x4<XT>(x, (size_t)t * H4 + c4);
+#pragma unroll
+                        for (int r = 0; r < RB; r++) {
+                            double a = acc[r][t];
+                            a = fma((double)xv.x, (double)wv[r][it].x, a);
+                            a = fma((double)xv.y, (double)wv[r][it].y, a);
+                            a = fma((double)xv.z, (double)wv[r][it].z, a);
+                            a = fma((double)xv.w, (double)wv[r][it].w, a);
+                            acc[r][t] = a;
+                        }
+                    }
                 }
             }
         }
@@ -171,8 +185,14 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     if (p.do_union) {
         __threadfence();
         __syncthreads();
-        union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status,
-                    smem);
+        if (p.T * p.k <= 32) {
+            if (warp == 0)
+                union_warp_small(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
+                                 p.status, lane);
+        } else {
+            union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
+                        p.status, smem);
+        }
     }
 }
 
@@ -253,6 +273,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const __grid_constant__ Route
 __global__ void __launch_bounds__(1024) union_kernel(const __grid_constant__ RouteParams p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
+    if (p.T * p.k <= 32) {
+        if (threadIdx.x < 32)
+            union_warp_small(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
+                             p.status, threadIdx.x);
+        return;
+    }
     union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status, smem);
 }
 
@@ -289,8 +315,8 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
 
 cudaError_t union_launch(const RouteParams& p, cudaStream_t s)
 {
-    const int nt = 1024;
-    const size_t smem = union_smem_bytes(p.E, nt / 32);
+    const int nt = (p.T * p.k <= 32) ? 32 : 1024;
+    const size_t smem = (p.T * p.k <= 32) ? 0 : union_smem_bytes(p.E, nt / 32);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
