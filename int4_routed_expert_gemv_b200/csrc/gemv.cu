@@ -53,6 +53,20 @@ __device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c)
     return (int32_t)d;
 }
 
+// Integer parts without the conversion unit: for |v| < 2^22, adding 1.5 * 2^23 leaves
+// the integer part of v (rounded in the requested direction) in the low mantissa bits.
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23, bits 0x4B400000
+__device__ __forceinline__ int floor_small(float v, float& fv)
+{
+    const float t = __fadd_rd(v, kMagic);
+    fv = t - kMagic;
+    return __float_as_int(t) - 0x4B400000;
+}
+__device__ __forceinline__ int rint_small(float v)
+{
+    return __float_as_int(__fadd_rn(v, kMagic)) - 0x4B400000;
+}
+
 // Activations of one 32-column unit as 8-bit digits.  With m = max |x_c| over the unit,
 // X_c = clamp(x_c * 126 / m, -126, 126) is written as
 //     X_c = a_c + b_c / 256 + c_c / 65536 + r_c,  a_c in [-126, 126] (signed),
@@ -91,11 +105,12 @@ __device__ __forceinline__ void load_digits(const float* src, uint32_t (&dg)[3][
 #pragma unroll
     for (int c = 0; c < 32; c++) {
         const float X = fminf(fmaxf(xv[c] * inv, -126.0f), 126.0f);
-        const float a = floorf(X);
+        float a, bq;
+        const int ai = floor_small(X, a);
         const float r1 = (X - a) * 256.0f;
-        const float bq = floorf(r1);
-        const float cq = fminf(rintf((r1 - bq) * 256.0f), 255.0f);
-        const int di[3] = {(int)a, (int)bq, (int)cq};
+        const int bi = floor_small(r1, bq);
+        const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
+        const int di[3] = {ai, bi, ci};
         const int wi = c >> 3, k = c & 7;
         const int slot = 2 * wi + (k & 1), byte = k >> 1;
 #pragma unroll
@@ -117,11 +132,12 @@ __device__ __forceinline__ void store_digit_record(float hv, int lane, uint32_t*
     for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     const float inv = mx > 0.0f ? 126.0f / mx : 0.0f;
     const float X = fminf(fmaxf(hv * inv, -126.0f), 126.0f);
-    const float a = floorf(X);
+    float a, bq;
+    const int ai = floor_small(X, a);
     const float r1 = (X - a) * 256.0f;
-    const float bq = floorf(r1);
-    const float cq = fminf(rintf((r1 - bq) * 256.0f), 255.0f);
-    const int di[3] = {(int)a, (int)bq, (int)cq};
+    const int bi = floor_small(r1, bq);
+    const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
+    const int di[3] = {ai, bi, ci};
     // lane L < 24 assembles word L: plane d = L / 8, slot s = L % 8
     const int d_me = lane >> 3, slot = lane & 7, wi = slot >> 1, par = slot & 1;
     uint32_t word = 0;

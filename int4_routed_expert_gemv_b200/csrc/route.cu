@@ -92,6 +92,42 @@ __device__ void topk_warp(const float* lt, int E, int k, int32_t* idx_t, float* 
     }
 }
 
+// Top-k of every token of a small batch by the whole block: thread i ranks pair
+// (t, e) = (i / E, i % E) against all E keys of its token in shared memory (keys are
+// unique, so ranks are a permutation); rank < k gives the slot.  Weights by one warp per
+// token.  smem: T*E keys (8 bytes) + T*k floats.
+__device__ void topk_block(const RouteParams& p, uint8_t* smem)
+{
+    uint64_t* skey = reinterpret_cast<uint64_t*>(smem);
+    float* ssel = reinterpret_cast<float*>(skey + (size_t)p.T * p.E);
+    const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5, lane = tid & 31;
+    const int TE = p.T * p.E;
+    for (int i = tid; i < TE; i += nt) {
+        const int t = i / p.E, e = i - t * p.E;
+        skey[i] = topk_key(__ldcg(p.logits + (size_t)t * p.E + e), e);
+    }
+    __syncthreads();
+    for (int i = tid; i < TE; i += nt) {
+        const int t = i / p.E;
+        const uint64_t* kt = skey + (size_t)t * p.E;
+        const uint64_t me = skey[i];
+        int rank = 0;
+#pragma unroll 8
+        for (int e2 = 0; e2 < p.E; e2++) rank += (kt[e2] > me) ? 1 : 0;
+        if (rank < p.k) {
+            p.idx[(size_t)t * p.k + rank] = i - t * p.E;
+            ssel[t * p.k + rank] = key_value(me);
+        }
+    }
+    __syncthreads();
+    for (int t = warp; t < p.T; t += nt / 32) {
+        double ex = 0.0;
+        if (lane < p.k) ex = exp((double)ssel[t * p.k + lane] - (double)ssel[t * p.k]);
+        const double z = dsum_warp(ex);
+        if (lane < p.k) p.w[(size_t)t * p.k + lane] = (float)(ex / z);
+    }
+}
+
 // Small batches: a CTA computes RB router rows for all T (<= kSmallT) tokens; threads
 // split the hidden dimension.  The last CTA to finish (ticket in the workspace header)
 // runs top-k for every token and, if asked, the batch union.
@@ -106,55 +142,47 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     const int H4 = p.H / 4;
     const XT* x = reinterpret_cast<const XT*>(p.x);
 
-    double acc[RB][kSmallT];
+    // token-outer: for each token every router and activation load of a pass is issued
+    // before the first FMA, so a pass costs one memory round trip (the second and later
+    // tokens find the CTA's router rows in L1)
+    constexpr int MAXIT = 8;   // one pass covers H <= 8192
+    for (int t = 0; t < p.T; t++) {
+        double acc[RB];
 #pragma unroll
-    for (int r = 0; r < RB; r++)
+        for (int r = 0; r < RB; r++) acc[r] = 0.0;
+        for (int base = 0; base < H4; base += 256 * MAXIT) {
+            float4 wv[RB][MAXIT], xv[MAXIT];
 #pragma unroll
-        for (int t = 0; t < kSmallT; t++) acc[r][t] = 0.0;
-    // all of this thread's router loads are issued before any arithmetic, so the CTA
-    // waits for one memory round trip per pass (one pass up to H = 8192)
-    constexpr int MAXIT = 8;
-    for (int base = 0; base < H4; base += 256 * MAXIT) {
-        float4 wv[RB][MAXIT];
+            for (int it = 0; it < MAXIT; it++) {
+                const int c4 = base + it * 256 + tid;
+                const bool in = c4 < H4;
 #pragma unroll
-        for (int it = 0; it < MAXIT; it++) {
-            const int c4 = base + it * 256 + tid;
+                for (int r = 0; r < RB; r++)
+                    wv[r][it] = (in && e0 + r < p.E)
+                                    ? __ldg(reinterpret_cast<const float4*>(p.w_router) +
+                                            (size_t)(e0 + r) * H4 + c4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                xv[it] = in ? load_x4<XT>(x, (size_t)t * H4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-            for (int r = 0; r < RB; r++)
-                wv[r][it] = (c4 < H4 && e0 + r < p.E)
-                                ? __ldcs(reinterpret_cast<const float4*>(p.w_router) +
-                                         (size_t)(e0 + r) * H4 + c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+            for (int it = 0; it < MAXIT; it++) {
 #pragma unroll
-        for (int it = 0; it < MAXIT; it++) {
-            const int c4 = base + it * 256 + tid;
-            if (c4 < H4) {
-#pragma unroll
-                for (int t = 0; t < kSmallT; t++) {
-                    if (t < p.T) {
-                        const float4 xv = load_x4<XT>(x, (size_t)t * H4 + c4);
-#pragma unroll
-                        for (int r = 0; r < RB; r++) {
-                            double a = acc[r][t];
-                            a = fma((double)xv.x, (double)wv[r][it].x, a);
-                            a = fma((double)xv.y, (double)wv[r][it].y, a);
-                            a = fma((double)xv.z, (double)wv[r][it].z, a);
-                            a = fma((double)xv.w, (double)wv[r][it].w, a);
-                            acc[r][t] = a;
-                        }
-                    }
+                for (int r = 0; r < RB; r++) {
+                    double a = acc[r];
+                    a = fma((double)xv[it].x, (double)wv[r][it].x, a);
+                    a = fma((double)xv[it].y, (double)wv[r][it].y, a);
+                    a = fma((double)xv[it].z, (double)wv[r][it].z, a);
+                    a = fma((double)xv[it].w, (double)wv[r][it].w, a);
+                    acc[r] = a;
                 }
             }
         }
-    }
 #pragma unroll
-    for (int r = 0; r < RB; r++)
-#pragma unroll
-        for (int t = 0; t < kSmallT; t++) {
-            const double v = dsum_warp(acc[r][t]);
+        for (int r = 0; r < RB; r++) {
+            const double v = dsum_warp(acc[r]);
             if (lane == 0) part[warp][r * kSmallT + t] = v;
         }
+    }
     __syncthreads();
     if (tid < RB * kSmallT) {
         const int r = tid / kSmallT, t = tid % kSmallT;
@@ -179,9 +207,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    for (int t = warp; t < p.T; t += 8)
-        topk_warp(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
-                  p.w + (size_t)t * p.k, lane);
+    topk_block(p, smem);
     if (p.do_union) {
         __threadfence();
         __syncthreads();
@@ -290,7 +316,9 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
     if (p.T <= kSmallT) {
         constexpr int RB = 2;
         const int grid = (p.E + RB - 1) / RB;
-        size_t smem = p.do_union ? union_smem_bytes(p.E, 8) : 0;
+        const size_t topk_smem = (size_t)p.T * p.E * 8 + (size_t)p.T * p.k * 4;
+        const size_t union_smem = (p.do_union && p.T * p.k > 32) ? union_smem_bytes(p.E, 8) : 0;
+        const size_t smem = topk_smem > union_smem ? topk_smem : union_smem;
         auto kern = bf16 ? router_small_kernel<__nv_bfloat16, RB> : router_small_kernel<float, RB>;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
