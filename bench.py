@@ -177,19 +177,27 @@ def run_ours(args, rank, world, local_rank):
         import dataclasses
         shp = dataclasses.replace(wl.shape, n_experts=args.n_experts)
         wl = dataclasses.replace(wl, shape=shp, name=f"{wl.name}_first{args.n_experts}experts")
-    if wl.layers != 1 or wl.x_dtype != "f32":
-        raise SystemExit(f"bench.py times single-layer fp32 workloads; got {wl.name}")
+    if wl.x_dtype != "f32":
+        raise SystemExit(f"bench.py times fp32 decode workloads; got {wl.name}")
     s = wl.shape
     T = wl.tokens
     H, I, E, k = s.hidden, s.inter, s.n_experts, s.top_k
+    NL = wl.layers
+    stack = NL > 1
 
-    experts = synth.experts_tensor(s, wl.seed, 0, device=dev)
-    shared = synth.shared_tensor(s, wl.seed, 0, device=dev)
-    wr = torch.from_numpy(synth.router_weight(s, wl.seed)).to(dev)
-    bias = torch.from_numpy(synth.zipf_bias(E)).to(dev) if wl.zipf else None
     dims = B.make_dims(H, I, E, k, s.n_shared)
-    weights = B.make_weights(wr, bias, experts, shared, s.stride)
+    layers = []
+    for l in range(NL):
+        ex = synth.experts_tensor(s, wl.seed, l, device=dev)
+        sh = synth.shared_tensor(s, wl.seed, l, device=dev)
+        wr = torch.from_numpy(synth.router_weight(s, wl.seed, l)).to(dev)
+        bias = torch.from_numpy(synth.zipf_bias(E)).to(dev) if wl.zipf else None
+        layers.append(dict(experts=ex, shared=sh, wr=wr, bias=bias,
+                           weights=B.make_weights(wr, bias, ex, sh, s.stride)))
     bufs = B.LayerBuffers(dims, T, device=dev)
+    gamma = torch.ones(H, dtype=torch.float32, device=dev)
+    x_work = torch.empty(T, H, dtype=torch.float32, device=dev)
+    n_work = torch.empty(T, H, dtype=torch.float32, device=dev)
 
     R = args.pool
     xs_host = [torch.from_numpy(synth.activations(s, wl.seed, T, 1000 + i)).pin_memory()
@@ -201,32 +209,53 @@ def run_ours(args, rank, world, local_rank):
     flush_read = torch.zeros(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
     flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    slots = 4 if stack else 3          # kernels timed per layer
 
-    # union size of every batch in the pool (deterministic), for the byte counts
-    n_union = []
-    for i in range(R):
-        B.check(B.coli_moe_route_union(dims, wr, bias, xs[i], T, bufs.idx, bufs.w, None,
+    def layer_calls(l, x_in, ev, e0):
+        """One layer; ev[e0 .. e0+slots] bracket its launches."""
+        L_ = layers[l]
+        if ev:
+            ev[e0].record()
+        if stack:
+            B.check(B.coli_rmsnorm(H, T, x_in, gamma, 1e-5, n_work), "rmsnorm")
+            if ev:
+                ev[e0 + 1].record()
+            act, res, y = n_work, x_in, x_in
+        else:
+            act, res, y = x_in, None, bufs.y
+        e = e0 + (1 if stack else 0)
+        B.check(B.coli_moe_route_union(dims, L_["wr"], L_["bias"], act, T, bufs.idx, bufs.w, None,
                                        bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
                                        bufs.ws), "route_union")
-        n_union.append(int(bufs.n_union[0].item()))
-
-    def step(i, ev=None):
-        x = xs[i % R]
         if ev:
-            ev[0].record()
-        B.check(B.coli_moe_route_union(dims, wr, bias, x, T, bufs.idx, bufs.w, None,
-                                       bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
-                                       bufs.ws), "route_union")
-        if ev:
-            ev[1].record()
-        B.check(B.coli_moe_gate_up(dims, weights, x, T, bufs.union_ids, bufs.n_union,
+            ev[e + 1].record()
+        B.check(B.coli_moe_gate_up(dims, L_["weights"], act, T, bufs.union_ids, bufs.n_union,
                                    bufs.offsets, bufs.assign, bufs.ws), "gate_up")
         if ev:
-            ev[2].record()
-        B.check(B.coli_moe_down(dims, weights, T, bufs.w, bufs.union_ids, bufs.n_union,
-                                bufs.offsets, bufs.assign, None, bufs.y, bufs.ws), "down")
+            ev[e + 2].record()
+        B.check(B.coli_moe_down(dims, L_["weights"], T, bufs.w, bufs.union_ids, bufs.n_union,
+                                bufs.offsets, bufs.assign, res, y, bufs.ws), "down")
         if ev:
-            ev[3].record()
+            ev[e + 3].record()
+
+    def step(i, ev=None):
+        if stack:
+            x_work.copy_(xs[i % R])
+            for l in range(NL):
+                layer_calls(l, x_work, ev, l * (slots + 1))
+        else:
+            layer_calls(0, xs[i % R], ev, 0)
+
+    # union size of every (batch, layer), deterministic, for the byte counts
+    n_union = []
+    for i in range(R):
+        row = []
+        if stack:
+            x_work.copy_(xs[i])
+        for l in range(NL):
+            layer_calls(l, x_work if stack else xs[i], None, 0)
+            row.append(int(bufs.n_union[0].item()))
+        n_union.append(row)
 
     def flush():
         # write 2x L2, then read another 2x L2: our data is evicted and L2 is left holding
@@ -234,10 +263,12 @@ def run_ours(args, rank, world, local_rank):
         flush_buf.zero_()
         torch.sum(flush_read, dim=0, keepdim=True, out=flush_sink)
 
-    # The timed steps run as CUDA graphs (flush + 3 launches per step, with event-record
+    # The timed steps run as CUDA graphs (flush + the step's launches, with event-record
     # nodes around each launch), so the GPU never waits for the host to enqueue work.
+    nev = NL * (slots + 1)
+
     def capture(first, n):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)]
                for _ in range(n)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -251,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
     sampler.start()
     time.sleep(0.2)
     K = args.steps
-    G = min(K, 128)
+    G = min(K, 128 if not stack else 8)
     chunks = [(c, min(G, K - c)) for c in range(0, K, G)]
     graphs = {}
     for (c, n) in chunks:
@@ -270,7 +301,13 @@ def run_ours(args, rank, world, local_rank):
         g, evs = graphs[n]
         g.replay()
         torch.cuda.synchronize(dev)
-        seg_rows += [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(n)]
+        for i in range(n):
+            per = np.zeros(slots)
+            for l in range(NL):
+                e0 = l * (slots + 1)
+                for j in range(slots):
+                    per[j] += evs[i][e0 + j].elapsed_time(evs[i][e0 + j + 1])
+            seg_rows.append(per)
     t1 = time.time()
     if world > 1:
         torch.distributed.barrier()
@@ -279,35 +316,44 @@ def run_ours(args, rank, world, local_rank):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     del graphs
-
     seg = np.array(seg_rows)
-    step_ms = seg.sum(axis=1)
+    if stack:
+        seg = seg[:, 1:]                 # route_union, gate_up, down (rmsnorm reported apart)
+        rms_ms = np.array(seg_rows)[:, 0]
+    step_ms = np.array(seg_rows).sum(axis=1)
     total_ms = float(step_ms.sum())
     st, bits = B.coli_moe_read_status(bufs.ws)
     if st != B.COLI_OK:
         raise SystemExit(f"device status {bits:#x} after the timed region")
 
-    # e2e: host buffers through the public layer call, copies inside the timed interval
+    # e2e: host buffers through the public calls, copies inside the timed interval
     e2e = None
     if not args.no_e2e:
         ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        xin = torch.empty_like(xs[0])
+
+        def e2e_step(i):
+            xin.copy_(xs_host[i % R], non_blocking=True)
+            if stack:
+                for l in range(NL):
+                    B.check(B.coli_rmsnorm(H, T, xin, gamma, 1e-5, n_work))
+                    B.check(B.coli_moe_layer(dims, layers[l]["weights"], n_work, T, bufs.idx,
+                                             bufs.w, None, bufs.union_ids, bufs.n_union,
+                                             bufs.offsets, bufs.assign, xin, xin, bufs.ws))
+                y_host.copy_(xin, non_blocking=True)
+            else:
+                B.check(B.coli_moe_layer(dims, layers[0]["weights"], xin, T, bufs.idx, bufs.w,
+                                         None, bufs.union_ids, bufs.n_union, bufs.offsets,
+                                         bufs.assign, None, bufs.y, bufs.ws))
+                y_host.copy_(bufs.y[:T], non_blocking=True)
         for i in range(min(args.warmup, 5)):
             flush()
-            xs[0].copy_(xs_host[i % R], non_blocking=True)
-            B.check(B.coli_moe_layer(dims, weights, xs[0], T, bufs.idx, bufs.w, None,
-                                     bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
-                                     None, bufs.y, bufs.ws))
-            y_host.copy_(bufs.y[:T], non_blocking=True)
+            e2e_step(i)
         torch.cuda.synchronize(dev)
-        xin = torch.empty_like(xs[0])
         for i in range(K):
             flush()
             ev2[i][0].record(stream)
-            xin.copy_(xs_host[i % R], non_blocking=True)
-            B.check(B.coli_moe_layer(dims, weights, xin, T, bufs.idx, bufs.w, None,
-                                     bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign,
-                                     None, bufs.y, bufs.ws))
-            y_host.copy_(bufs.y[:T], non_blocking=True)
+            e2e_step(i)
             ev2[i][1].record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = float(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(K)))
@@ -320,22 +366,22 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
 
-    # algorithmic bytes
+    # algorithmic bytes (per step, summed over the layers of the step)
     blob = s.blob_bytes
     gu_bytes_expert = 2 * (I * H // 2) + 2 * (I * H // 64) * 2
     dn_bytes_expert = H * I // 2 + H * (I // 64) * 2
-    nu = np.array([n_union[(args.warmup + i) % R] for (c, n) in chunks for i in range(n)],
+    nu = np.array([sum(n_union[(args.warmup + i) % R]) for (c, n) in chunks for i in range(n)],
                   dtype=np.float64)
-    units = nu + s.n_shared
+    units = nu + NL * s.n_shared
     x_bytes = T * H * 4
     h_bytes = (T * k + T * s.n_shared) * I * 4
-    route_bytes = E * H * 4 + x_bytes + T * E * 4
-    gu_bytes = units * gu_bytes_expert + x_bytes + h_bytes
-    dn_bytes = units * dn_bytes_expert + h_bytes + T * H * 4
-    step_bytes = route_bytes + units * blob + x_bytes + 2 * h_bytes + T * H * 4
+    route_bytes = NL * (E * H * 4 + x_bytes + T * E * 4)
+    gu_bytes = units * gu_bytes_expert + NL * (x_bytes + h_bytes)
+    dn_bytes = units * dn_bytes_expert + NL * (h_bytes + T * H * 4)
+    step_bytes = route_bytes + units * blob + NL * (x_bytes + 2 * h_bytes + T * H * 4)
     peak, peak_kind = measured_peaks()
     kern = {
-        "route_union": (seg[:, 0], np.full(K, route_bytes)),
+        "route_union": (seg[:, 0], np.full(K, float(route_bytes))),
         "gate_up": (seg[:, 1], gu_bytes),
         "down": (seg[:, 2], dn_bytes),
     }
@@ -346,11 +392,14 @@ def run_ours(args, rank, world, local_rank):
         kernels[name] = {"avg_us": round(avg_ms * 1e3, 3), "bytes_per_launch": float(by.mean()),
                          "gb_s": round(gbs, 1), "frac": round(gbs / peak, 4),
                          "share": round(float(ms.sum() / seg.sum()), 4)}
-    dom = max(kernels, key=lambda n: kernels[n]["share"])
+    if stack:
+        kernels["rmsnorm"] = {"avg_us": round(float(rms_ms.mean()) * 1e3, 3),
+                              "share": round(float(rms_ms.sum() / step_ms.sum()), 4)}
+    dom = max((n for n in kernels if n != "rmsnorm"), key=lambda n: kernels[n]["share"])
     traffic = recorded_traffic(dom, wl.name)
     tokens = T * K * world
     value = tokens / (total_ms * 1e-3)
-    launches_per_step = (1 if T <= 8 else 3) + 2
+    launches_per_step = NL * ((1 if T <= 8 else 3) + 2 + (1 if stack else 0))
 
     out = {
         "metric": METRIC,
@@ -365,13 +414,14 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "tokens_per_step": T, "hidden": H, "intermediate": I,
+        "config": {"workload": wl.name, "tokens_per_step": T, "layers": NL, "hidden": H,
+                   "intermediate": I,
                    "experts": E, "top_k": k, "shared_experts": s.n_shared,
                    "weights": "gs64 int4, fp16 scales", "activations": "fp32",
                    "l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
                    "timing": "CUDA graphs of up to 128 steps; events around each launch",
                    "token_pool": R, "parallelism": f"replicas x{world}",
-                   "mean_union": float(nu.mean())},
+                   "mean_union_per_layer": float(nu.mean() / NL)},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gb_s"],
                      "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "unit": "GB/s", "frac": kernels[dom]["frac"],
@@ -387,7 +437,9 @@ def run_ours(args, rank, world, local_rank):
         out["e2e"] = {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
                       "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2],
                       "api": "coli_moe_layer with pinned-host x in and y out"}
-    if world == 1 and not args.no_cpu_baseline:
+    if stack:
+        out["config"]["kernel_figures"] = f"per step (sum over the {NL} layers' launches)"
+    if world == 1 and not args.no_cpu_baseline and not stack:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     return out
 

@@ -70,8 +70,9 @@ __device__ __forceinline__ int rint_small(float v)
 // Activations of one 32-column unit as 8-bit digits.  With m = max |x_c| over the unit,
 // X_c = clamp(x_c * 126 / m, -126, 126) is written as
 //     X_c = a_c + b_c / 256 + c_c / 65536 + r_c,  a_c in [-126, 126] (signed),
-//     b_c, c_c in [0, 255] (unsigned),  0 <= r_c < 2^-16
-// (floor digits, the last one rounded), so that
+//     b_c, c_c in [0, 255] (unsigned),  |r_c| <= 2^-16
+// (floor digits, the last one rounded; when X_c - a_c rounds to 1.0f for a tiny negative
+// X_c the middle digit saturates at 255), so that
 //     sum_c q_c x_c = (m / (126 * 65536)) * sum_c q_c (65536 a_c + 256 b_c + c_c)
 // up to about 1.2e-7 m per column, with the integer sum exact in int32 (below 2^31 for
 // |q| <= 8 over 32 columns).  Weight nibbles arrive in offset binary n' = q + 8, so each
@@ -107,8 +108,14 @@ __device__ __forceinline__ void load_digits(const float* src, uint32_t (&dg)[3][
         const float X = fminf(fmaxf(xv[c] * inv, -126.0f), 126.0f);
         float a, bq;
         const int ai = floor_small(X, a);
+        // X - a can round up to exactly 1.0f when X is a tiny negative number; the second
+        // digit then saturates at 255 and the third absorbs the remainder
         const float r1 = (X - a) * 256.0f;
-        const int bi = floor_small(r1, bq);
+        int bi = floor_small(r1, bq);
+        if (bi > 255) {
+            bi = 255;
+            bq = 255.0f;
+        }
         const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
         const int di[3] = {ai, bi, ci};
         const int wi = c >> 3, k = c & 7;
@@ -134,8 +141,12 @@ __device__ __forceinline__ void store_digit_record(float hv, int lane, uint32_t*
     const float X = fminf(fmaxf(hv * inv, -126.0f), 126.0f);
     float a, bq;
     const int ai = floor_small(X, a);
-    const float r1 = (X - a) * 256.0f;
-    const int bi = floor_small(r1, bq);
+    const float r1 = (X - a) * 256.0f;       // may be exactly 256 for tiny negative X
+    int bi = floor_small(r1, bq);
+    if (bi > 255) {
+        bi = 255;
+        bq = 255.0f;
+    }
     const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
     const int di[3] = {ai, bi, ci};
     // lane L < 24 assembles word L: plane d = L / 8, slot s = L % 8

@@ -182,3 +182,16 @@ def test_rmsnorm_matches_oracle():
     ref = oracle.rmsnorm(x, g, 1e-5)
     got = out.cpu().numpy()
     assert np.max(np.abs(got.view(np.int32) - ref.view(np.int32))) <= 1
+
+
+@pytest.mark.parametrize("scale", [4.0, 16.0])
+def test_large_activations_tiny_negative_h(scale):
+    # large x drives many gate values far negative: silu(g) * u is then a tiny negative
+    # number, the case where a floor-digit split of h can round up to the next integer
+    shape = synth.LayerShape(1024, 512, 64, 4, 1)
+    L = make_device_layer(shape, 13)
+    x = (synth.activations(shape, 13, 3, 2) * scale).astype(np.float32)
+    got = run_layer(L, torch.from_numpy(x).cuda(), 3)
+    ref = oracle_layer(L, x)
+    assert_route_union_equal(got, ref)
+    assert_y_close(got["y"], ref["y"], rel_l2=1e-5)
