@@ -115,7 +115,10 @@ def blob_weight(H, I, blob, which, r, c, bf16=False) -> float:
 
 
 def expert(H, I, blob, x, bf16=False):
-    """One expert on one token -> (out [H] float64, h [I] float64)."""
+    """One expert on one token -> (out [H] float64, h [I] float64).
+
+    bf16: False/0 fp32 contract; True/1 bf16 weights and bf16 h; 2 bf16 weights, exact h.
+    """
     blob = _c(blob, np.uint8)
     x = _c(x, np.float32)
     out = np.zeros(H, np.float64)

@@ -42,10 +42,14 @@
  * Precision modes of the expert FFN:
  *   mode 0 (fp32 contract): weights are q*scale exactly, activations as given, all sums
  *           in double, h kept in double, y rounded once to float.
- *   mode 1 (bf16 contract, used by the tensor-core prefill path): every dequantised
- *           weight q*scale is rounded to bfloat16 (round-to-nearest-even) before use, and
- *           h = silu(g)*u is rounded to float and then to bfloat16 before the down
- *           projection.  Sums stay in double.
+ *   mode 1 (bf16 weights and bf16 h): every dequantised weight q*scale is rounded to
+ *           bfloat16 (round-to-nearest-even) before use, and h = silu(g)*u is rounded to
+ *           float and then to bfloat16 before the down projection.  Sums stay in double.
+ *   mode 2 (bf16 weights, exact h): weights rounded to bfloat16 as in mode 1, h kept in
+ *           double.  This is the contract of the tensor-core prefill path, which carries h
+ *           into the down projection as a pair of bfloat16 values (about 16 significant
+ *           bits) so that no rounding decision on h has to agree between two
+ *           implementations that compute g and u in different precisions.
  */
 #include <math.h>
 #include <stdint.h>
@@ -187,7 +191,7 @@ int orc_expert(int H, int I, const uint8_t *blob, const float *x, int bf16, doub
         for (int64_t c = 0; c < H; c++)
             u += weight(v.uq, v.us, H, i, c, bf16) * (double)x[c];
         double hi = silu(g) * u;
-        if (bf16)
+        if (bf16 == 1)
             hi = (double)orc_bf16_round((float)hi);
         h[i] = hi;
         if (h_out)

@@ -406,3 +406,26 @@ def test_rmsnorm_closed_form_and_numpy():
     x64 = x.astype(np.float64)
     ref = x64 / np.sqrt(np.mean(x64 ** 2, axis=1, keepdims=True) + 1e-5) * gmm
     assert np.allclose(out, ref, rtol=2 ** -23, atol=0)
+
+
+def test_bf16_weights_exact_h_mode():
+    # mode 2 rounds only the weights: with bf16-representable weights it equals the fp32
+    # contract exactly, and it differs from mode 1 exactly by the rounding of h
+    H = I = 64
+    rng = np.random.default_rng(11)
+    q = [rng.integers(-8, 8, s) for s in [(I, H), (I, H), (H, I)]]
+    s = [np.full((I, 1), 2.0 ** -6, np.float16), np.full((I, 1), 2.0 ** -5, np.float16),
+         np.full((H, 1), 2.0 ** -7, np.float16)]
+    blob = make_blob(q[0], s[0], q[1], s[1], q[2], s[2])
+    x = torch.from_numpy(rng.standard_normal(H).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    out0, h0 = oracle.expert(H, I, blob, x, bf16=0)
+    out2, h2 = oracle.expert(H, I, blob, x, bf16=2)
+    out1, h1 = oracle.expert(H, I, blob, x, bf16=1)
+    assert np.array_equal(out0, out2) and np.array_equal(h0, h2)
+    assert not np.array_equal(h1, h2)
+    assert np.array_equal(h1, torch.from_numpy(h2.astype(np.float32)).to(torch.bfloat16).double().numpy())
+    # non-representable weights: mode 2 uses the rounded weights, like mode 1
+    blob, dense = random_expert(rng, H, I)
+    for r, c in [(0, 0), (5, 63), (63, 1)]:
+        assert (oracle.blob_weight(H, I, blob, 0, r, c, bf16=2) ==
+                oracle.blob_weight(H, I, blob, 0, r, c, bf16=1))
