@@ -32,8 +32,9 @@
  *   COLI_F32  decode GEMV path: weights are applied exactly (q * scale in fp32), all
  *             products and sums in fp32 (routing in fp64), h kept in fp32.
  *   COLI_BF16 prefill path: x is bf16; every dequantised weight is rounded to bf16
- *             (nearest-even), products accumulate in fp32 on the tensor cores, and h is
- *             rounded to bf16 before the down projection.  Routing stays fp64/fp32.
+ *             (nearest-even), products accumulate in fp32 on the tensor cores, and h
+ *             enters the down projection as a pair of bf16 values (hi = bf16(h),
+ *             lo = bf16(h - hi), about 16 significant bits).  Routing stays fp64/fp32.
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller, 16-byte aligned,
