@@ -20,13 +20,13 @@
 // significant bits; the two halves' MMAs accumulate into the same tensor-memory tile), so
 // no result depends on where a bf16 rounding of h falls.
 //
-// CTA (one per SM, persistent over a static share of the task list), 10 warps:
-//   warps 0-3  epilogue: tcgen05.ld of the accumulators, SwiGLU or the weighted combine
-//   warps 4-7  dequantisers: thread r turns row r of the raw int4 tile (TMA-staged) into
-//              bf16 and writes it 128B-swizzled into the A tile
-//   warp 8     TMA producer: raw nibble rows (3-D tensor map over all experts) and the
-//              token tile (2-D tensor map, 128B swizzle)
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+// CTA (one per SM, persistent over a static share of the task list), 14 warps:
+//   warps 0-3   epilogue: tcgen05.ld of the accumulators, SwiGLU or the weighted combine
+//   warps 4-11  dequantisers: threads 2r and 2r+1 turn the two halves of row r of the raw
+//               int4 tile (TMA-staged) into bf16, written 128B-swizzled into the A tile
+//   warp 12     TMA producer: raw nibble rows (3-D tensor map over all experts) and the
+//               token tiles (2-D tensor maps, 128B swizzle)
+//   warp 13     TMEM allocator and single-thread tcgen05.mma issuer
 // Accumulators are double-buffered in tensor memory so a task's epilogue overlaps the
 // next task's MMAs.  Every mbarrier wait is bounded (DEV_TIMEOUT, then no more waiting).
 #include <cuda.h>
@@ -42,7 +42,7 @@ namespace {
 constexpr int kRows = 128;        // weight rows per tile (MMA M)
 constexpr int kKc = 64;           // K per pipeline stage (one scale group)
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kNmax0 = 128;       // tokens per task, gate/up (G and U accumulators)
 constexpr int kNmax1 = 128;       // tokens per task, down (h as a hi + lo pair)
 constexpr int kNumBoxes = 5;      // token-tile heights 16, 32, 64, 128, 256
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     if (tid == 0) {
         for (int s = 0; s < kStages; s++) {
             mbar_init(&full_in[s], 1);
-            mbar_init(&a_full[s], 4);          // one arrival per dequant warp
+            mbar_init(&a_full[s], 8);          // one arrival per dequant warp
             mbar_init(&empty[s], 1);           // MMA commit
         }
         for (int b = 0; b < 2; b++) {
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         mbar_init(mma_done, 1);
         fence_barrier_init();
     }
-    if (warp == 9) tmem_alloc(tmem_base_smem, 512);
+    if (warp == 13) tmem_alloc(tmem_base_smem, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     // stage layout: A tiles (nmat x 16 KB) | token tile | raw tiles (nmat x 4 KB)
     bool dead = false;
 
-    if (warp == 8) {
+    if (warp == 12) {
         // ---------------------------------- TMA producer ------------------------------
         if (lane == 0) {
             uint32_t it = 0;
@@ -320,9 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 mbar_wait(&full_in[last % kStages], (last / kStages) & 1, p.status, kWaitSite + 2);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ---------------------------------- dequantisers ------------------------------
-        const int r = tid - 128;               // weight row within the 128-row tile
+        const int r = (tid - 128) >> 1;        // weight row within the 128-row tile
+        const int half = (tid - 128) & 1;      // 16-byte chunks 4*half .. 4*half+3 of the row
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntasks; t += gridDim.x) {
             const Task tk = p.tasks[t];
@@ -345,15 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 for (int mt = 0; mt < nmat; mt++) {
                     const float sc = __half2float(__ushort_as_half(__ldg(srow[mt] + kc)));
                     const uint64_t sp = pk2f(sc, sc);
-                    const uint4* rw = reinterpret_cast<const uint4*>(st + nmat * a_bytes + b_bytes +
-                                                                     mt * raw_bytes + r * 32);
-                    const uint4 w0 = rw[0], w1 = rw[1];
-                    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(st + nmat * a_bytes + b_bytes +
+                                                                     mt * raw_bytes + r * 32 + half * 16);
+                    const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
                     uint8_t* arow = st + mt * a_bytes + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-                    for (int c = 0; c < 8; c++) {        // 16-byte chunk c = columns 8c .. 8c+7
+                    for (int c4 = 0; c4 < 4; c4++) {     // 16-byte chunk c = columns 8c .. 8c+7
+                        const int c = 4 * half + c4;
                         uint32_t o[4];
-                        dq8_bf16(words[c], sp, o);
+                        dq8_bf16(words[c4], sp, o);
                         *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 if (lane == 0) mbar_arrive(&a_full[s]);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // ---------------------------------- MMA issuer --------------------------------
         if (lane == 0) {
             uint32_t it = 0, tcount = 0;
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             umma_commit(mma_done);
             mbar_wait(mma_done, 0, p.status, kWaitSite + 8);
         }
-    } else {
+    } else if (warp < 4) {
         // ---------------------------------- epilogue ----------------------------------
         const int q = warp;                    // TMEM lane quarter
         const int row = q * 32 + lane;         // weight row within the tile
@@ -421,8 +422,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 uint32_t g[16], u[16];
                 tmem_ld16(lane_addr + (uint32_t)c0, g);
                 if (phase == 0) tmem_ld16(lane_addr + 128u + (uint32_t)c0, u);
-                tmem_wait_ld();
                 const int nc = min(16, tk.ntok - c0);
+                // phase 1: lane j < nc fetches token c0 + j's id and routing weight once
+                int my_tok = 0;
+                float my_w = 0.0f;
+                if (phase == 1 && lane < nc) {
+                    const int tt = tk.tok0 + c0 + lane;
+                    if (sv.expert < 0) {
+                        my_tok = tt;
+                        my_w = 1.0f;
+                    } else {
+                        const int a = p.assign[sv.base + tt];
+                        my_tok = a / p.k;
+                        my_w = p.w[a];
+                    }
+                }
+                tmem_wait_ld();
                 for (int j = 0; j < nc; j++) {
                     const int tt = tk.tok0 + c0 + j;      // token index within the segment
                     if (phase == 0) {
@@ -433,16 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                         p.h[o] = hh;
                         p.h_lo[o] = __float2bfloat16_rn(hv - __bfloat162float(hh));
                     } else {
-                        int tok;
-                        float wt;
-                        if (sv.expert < 0) {
-                            tok = tt;
-                            wt = 1.0f;
-                        } else {
-                            const int a = p.assign[sv.base + tt];
-                            tok = a / p.k;
-                            wt = p.w[a];
-                        }
+                        const int tok = __shfl_sync(0xffffffffu, my_tok, j);
+                        const float wt = __shfl_sync(0xffffffffu, my_w, j);
                         atomicAdd(p.y + (size_t)tok * p.H + grow, wt * __uint_as_float(g[j]));
                     }
                 }
@@ -454,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

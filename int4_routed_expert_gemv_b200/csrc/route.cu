@@ -222,61 +222,49 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     }
 }
 
-// Large batches: 64 tokens x 64 experts per CTA, 32-column slabs staged in shared
-// memory, each thread accumulates 4 x 4 logits in double.
+// Large batches: 32 tokens x 32 experts per CTA, 32-column slabs converted to double once
+// when staged in shared memory; each thread accumulates 2 x 2 logits in double.
 template <typename XT>
 __global__ void __launch_bounds__(256) router_tiled_kernel(const __grid_constant__ RouteParams p)
 {
-    __shared__ float xs[32][64 + 4];
-    __shared__ float ws[32][64 + 4];
+    __shared__ __align__(16) double xs[32][34];   // [k][token]
+    __shared__ __align__(16) double ws[32][34];   // [k][expert]
     const int tid = threadIdx.x;
-    const int t0 = blockIdx.y * 64, e0 = blockIdx.x * 64;
+    const int t0 = blockIdx.y * 32, e0 = blockIdx.x * 32;
     const int ty = tid / 16, tx = tid % 16;
     const XT* x = reinterpret_cast<const XT*>(p.x);
-    double acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; a++)
-#pragma unroll
-        for (int b = 0; b < 4; b++) acc[a][b] = 0.0;
+    double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+    const int row = tid / 8, c4 = tid % 8;        // staging: 32 rows x 8 float4
     for (int k0 = 0; k0 < p.H; k0 += 32) {
-        // 64 rows x 32 columns of x and of W_r: 512 float4 each, 2 per thread
-#pragma unroll
-        for (int q = 0; q < 2; q++) {
-            const int f = tid + 256 * q;
-            const int row = f / 8, c4 = f % 8;
-            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
-            if (t0 + row < p.T) xv = load_x4<XT>(x, ((size_t)(t0 + row) * p.H + k0) / 4 + c4);
-            if (e0 + row < p.E)
-                wv = __ldg(reinterpret_cast<const float4*>(p.w_router) +
-                           ((size_t)(e0 + row) * p.H + k0) / 4 + c4);
-            xs[c4 * 4 + 0][row] = xv.x;
-            xs[c4 * 4 + 1][row] = xv.y;
-            xs[c4 * 4 + 2][row] = xv.z;
-            xs[c4 * 4 + 3][row] = xv.w;
-            ws[c4 * 4 + 0][row] = wv.x;
-            ws[c4 * 4 + 1][row] = wv.y;
-            ws[c4 * 4 + 2][row] = wv.z;
-            ws[c4 * 4 + 3][row] = wv.w;
-        }
+        float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
+        if (t0 + row < p.T) xv = load_x4<XT>(x, ((size_t)(t0 + row) * p.H + k0) / 4 + c4);
+        if (e0 + row < p.E)
+            wv = __ldg(reinterpret_cast<const float4*>(p.w_router) + ((size_t)(e0 + row) * p.H + k0) / 4 + c4);
+        __syncthreads();
+        xs[c4 * 4 + 0][row] = xv.x;
+        xs[c4 * 4 + 1][row] = xv.y;
+        xs[c4 * 4 + 2][row] = xv.z;
+        xs[c4 * 4 + 3][row] = xv.w;
+        ws[c4 * 4 + 0][row] = wv.x;
+        ws[c4 * 4 + 1][row] = wv.y;
+        ws[c4 * 4 + 2][row] = wv.z;
+        ws[c4 * 4 + 3][row] = wv.w;
         __syncthreads();
 #pragma unroll 8
         for (int kk = 0; kk < 32; kk++) {
-            const float4 a4 = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-            const float4 b4 = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-            const double a[4] = {a4.x, a4.y, a4.z, a4.w};
-            const double b[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-            for (int i = 0; i < 4; i++)
-#pragma unroll
-                for (int jj = 0; jj < 4; jj++) acc[i][jj] = fma(a[i], b[jj], acc[i][jj]);
+            const double2 a = *reinterpret_cast<const double2*>(&xs[kk][ty * 2]);
+            const double2 b = *reinterpret_cast<const double2*>(&ws[kk][tx * 2]);
+            acc[0][0] = fma(a.x, b.x, acc[0][0]);
+            acc[0][1] = fma(a.x, b.y, acc[0][1]);
+            acc[1][0] = fma(a.y, b.x, acc[1][0]);
+            acc[1][1] = fma(a.y, b.y, acc[1][1]);
         }
-        __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; i++)
+    for (int i = 0; i < 2; i++)
 #pragma unroll
-        for (int jj = 0; jj < 4; jj++) {
-            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + jj;
+        for (int jj = 0; jj < 2; jj++) {
+            const int t = t0 + ty * 2 + i, e = e0 + tx * 2 + jj;
             if (t < p.T && e < p.E) {
                 double s = acc[i][jj];
                 if (p.bias) s += (double)p.bias[e];
@@ -328,7 +316,7 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
         kern<<<grid, 256, smem, s>>>(p);
         return cudaGetLastError();
     }
-    dim3 grid((p.E + 63) / 64, (p.T + 63) / 64);
+    dim3 grid((p.E + 31) / 32, (p.T + 31) / 32);
     if (bf16)
         router_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
     else
