@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--n-experts", type=int, default=0,
                     help="profiling captures only: keep the first N routed experts")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling captures only: tokens per step instead of the workload's")
     return ap.parse_args()
 
 
@@ -177,6 +179,9 @@ def run_ours(args, rank, world, local_rank):
         import dataclasses
         shp = dataclasses.replace(wl.shape, n_experts=args.n_experts)
         wl = dataclasses.replace(wl, shape=shp, name=f"{wl.name}_first{args.n_experts}experts")
+    if args.tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, tokens=args.tokens, name=f"{wl.name}_as_t{args.tokens}")
     if wl.x_dtype == "bf16":
         return run_prefill(args, wl, rank, world, dev)
     s = wl.shape

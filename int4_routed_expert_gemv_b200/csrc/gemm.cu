@@ -438,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                     }
                 }
                 tmem_wait_ld();
-                for (int j = 0; j < nc; j++) {
+#pragma unroll
+                for (int j = 0; j < 16; j++) {            // unrolled: g, u stay in registers
+                    if (j >= nc) break;
                     const int tt = tk.tok0 + c0 + j;      // token index within the segment
                     if (phase == 0) {
                         const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
