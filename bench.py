@@ -251,6 +251,18 @@ def run_ours(args, rank, world, local_rank):
         else:
             layer_calls(0, xs[i % R], ev, 0)
 
+    def step_coarse(i, ev):
+        """The same launches with events only around the whole step (no event nodes between
+        kernels, so consecutive launches keep their programmatic dependency)."""
+        ev[0].record()
+        if stack:
+            x_work.copy_(xs[i % R])
+            for l in range(NL):
+                layer_calls(l, x_work, None, 0)
+        else:
+            layer_calls(0, xs[i % R], None, 0)
+        ev[1].record()
+
     # union size of every (batch, layer), deterministic, for the byte counts
     n_union = []
     for i in range(R):
@@ -272,14 +284,17 @@ def run_ours(args, rank, world, local_rank):
     # nodes around each launch), so the GPU never waits for the host to enqueue work.
     nev = NL * (slots + 1)
 
-    def capture(first, n):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)]
+    def capture(first, n, coarse=False):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 if coarse else nev)]
                for _ in range(n)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(n):
                 flush()
-                step(first + i, evs[i])
+                if coarse:
+                    step_coarse(first + i, evs[i])
+                else:
+                    step(first + i, evs[i])
         return g, evs
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -292,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
     graphs = {}
     for (c, n) in chunks:
         if n not in graphs:
-            graphs[n] = capture(args.warmup, n)
+            graphs[n] = capture(args.warmup, n, coarse=True)
     if args.warmup:
         gw, _ = capture(0, args.warmup)
         gw.replay()
@@ -300,32 +315,43 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    seg_rows = []
+    # timed: K steps, events around each whole step (the flush stays outside)
+    step_rows = []
     t0 = time.time()
     for (c, n) in chunks:
         g, evs = graphs[n]
         g.replay()
         torch.cuda.synchronize(dev)
         for i in range(n):
-            per = np.zeros(slots)
-            for l in range(NL):
-                e0 = l * (slots + 1)
-                for j in range(slots):
-                    per[j] += evs[i][e0 + j].elapsed_time(evs[i][e0 + j + 1])
-            seg_rows.append(per)
+            step_rows.append(evs[i][0].elapsed_time(evs[i][1]))
     t1 = time.time()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
+    del graphs
+    # per-kernel breakdown (for the roofline): the same steps with an event around every
+    # launch; these events serialise the launches, so their sum is a little above the step
+    Kb = min(K, G)
+    gb, evb = capture(args.warmup, Kb)
+    gb.replay()
+    torch.cuda.synchronize(dev)
+    seg_rows = []
+    for i in range(Kb):
+        per = np.zeros(slots)
+        for l in range(NL):
+            e0 = l * (slots + 1)
+            for j in range(slots):
+                per[j] += evb[i][e0 + j].elapsed_time(evb[i][e0 + j + 1])
+        seg_rows.append(per)
+    del gb
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
-    del graphs
     seg = np.array(seg_rows)
     if stack:
         seg = seg[:, 1:]                 # route_union, gate_up, down (rmsnorm reported apart)
         rms_ms = np.array(seg_rows)[:, 0]
-    step_ms = np.array(seg_rows).sum(axis=1)
+    step_ms = np.array(step_rows)
     total_ms = float(step_ms.sum())
     st, bits = B.coli_moe_read_status(bufs.ws)
     if st != B.COLI_OK:
@@ -386,9 +412,9 @@ def run_ours(args, rank, world, local_rank):
     step_bytes = route_bytes + units * blob + NL * (x_bytes + 2 * h_bytes + T * H * 4)
     peak, peak_kind = measured_peaks()
     kern = {
-        "route_union": (seg[:, 0], np.full(K, float(route_bytes))),
-        "gate_up": (seg[:, 1], gu_bytes),
-        "down": (seg[:, 2], dn_bytes),
+        "route_union": (seg[:, 0], np.full(Kb, float(route_bytes))),
+        "gate_up": (seg[:, 1], gu_bytes[:Kb]),
+        "down": (seg[:, 2], dn_bytes[:Kb]),
     }
     kernels = {}
     for name, (ms, by) in kern.items():
@@ -424,7 +450,8 @@ def run_ours(args, rank, world, local_rank):
                    "experts": E, "top_k": k, "shared_experts": s.n_shared,
                    "weights": "gs64 int4, fp16 scales", "activations": "fp32",
                    "l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
-                   "timing": "CUDA graphs of up to 128 steps; events around each launch",
+                   "timing": "CUDA graphs of up to 128 steps; events around each step (the value); "
+                             "per-kernel figures from a second pass with events around each launch",
                    "token_pool": R, "parallelism": f"replicas x{world}",
                    "mean_union_per_layer": float(nu.mean() / NL)},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gb_s"],

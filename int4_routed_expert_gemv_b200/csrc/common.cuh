@@ -128,6 +128,16 @@ __device__ __forceinline__ void bulk_g2s_hint(void* smem_dst, const void* gsrc, 
         : "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the stream
+// (launched with programmatic stream serialization) be scheduled before this one ends;
+// wait blocks until the kernels this one depends on have completed and their memory is
+// visible.  Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Named barrier over a subset of warps (id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads)
 {

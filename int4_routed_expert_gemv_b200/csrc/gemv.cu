@@ -36,6 +36,7 @@ namespace {
 constexpr int kBarFull = 0;      // mbarrier slots in shared memory
 constexpr int kMaxStages = 16;
 constexpr int kMaxChunks = 64;      // pending chunks per flush
+constexpr int kVecBufs = 4;         // activation (x or h digit record) buffers when not resident
 
 // dp4a: c + sum_i a_i * b_i over the four bytes, exact in 32-bit integers; a's bytes
 // unsigned, b's bytes signed (dp4a_us) or unsigned (dp4a_uu, wrapping mod 2^32)
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     uint64_t* vfull = empty + kMaxStages;
-    uint64_t* vempty = vfull + 2;
+    uint64_t* vempty = vfull + kVecBufs;
     float* red = reinterpret_cast<float*>(smem + p.off_red);
     uint8_t* vec = smem + p.off_vec;
     uint8_t* stages = smem + p.off_stage;
@@ -316,21 +317,25 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int K = p.K;
-    const int nu = *p.n_union;
-    const int nseg = p.n_shared + nu;
+    pdl_launch_dependents();
 
     if (tid == 0) {
         for (int s = 0; s < p.NS; s++) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NCONS / 32);
         }
-        for (int b = 0; b < 2; b++) {
+        for (int b = 0; b < kVecBufs; b++) {
             mbar_init(&vfull[b], 1);
             mbar_init(&vempty[b], NCONS / 32);
         }
         fence_barrier_init();
     }
     __syncthreads();
+    // everything above overlaps the previous kernel; routing, activations and h are read
+    // only after it has completed
+    pdl_wait();
+    const int nu = *p.n_union;
+    const int nseg = p.n_shared + nu;
 
     if (warp == NCONS / 32) {
         // ------------------------------- producer ------------------------------------
@@ -348,8 +353,8 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             for (int c0 = 0; c0 < g.count; c0 += MAXM) {
                 const int M = min(MAXM, g.count - c0);
                 if (!p.resident) {
-                    const int b = vit & 1;
-                    if (!dead && !mbar_wait(&vempty[b], ((vit >> 1) & 1) ^ 1, p.status, 11))
+                    const int b = vit % kVecBufs;
+                    if (!dead && !mbar_wait(&vempty[b], ((vit / kVecBufs) & 1) ^ 1, p.status, 11))
                         dead = true;
                     if (!dead) {
                         uint8_t* dst = vec + b * p.vec_bytes;
@@ -404,9 +409,9 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             mbar_wait(&full[last % p.NS], (last / p.NS) & 1, p.status, 13);
         }
         if (!p.resident) {
-            for (uint32_t q = 0; q < (vit < 2u ? vit : 2u); q++) {
+            for (uint32_t q = 0; q < (vit < (uint32_t)kVecBufs ? vit : (uint32_t)kVecBufs); q++) {
                 const uint32_t last = vit - 1 - q;
-                mbar_wait(&vfull[last & 1], (last >> 1) & 1, p.status, 14);
+                mbar_wait(&vfull[last % kVecBufs], (last / kVecBufs) & 1, p.status, 14);
             }
         } else {
             mbar_wait(&vfull[0], 0, p.status, 15);
@@ -532,8 +537,8 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             const float* vsrc;
             int b = 0;
             if (!p.resident) {
-                b = vit & 1;
-                if (!dead && !mbar_wait(&vfull[b], (vit >> 1) & 1, p.status, 22)) dead = true;
+                b = vit % kVecBufs;
+                if (!dead && !mbar_wait(&vfull[b], (vit / kVecBufs) & 1, p.status, 22)) dead = true;
                 vsrc = reinterpret_cast<const float*>(vec + b * p.vec_bytes);
             } else {
                 vsrc = reinterpret_cast<const float*>(vec);
@@ -695,8 +700,19 @@ cudaError_t launch_one(const GemvParams& p, const GemvConfig& c, cudaStream_t s)
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) set_bytes[dev] = (int)c.smem;
     }
-    kern<<<c.grid, c.consumers + 32, c.smem, s>>>(p);
-    return cudaGetLastError();
+    // programmatic stream serialization: the kernel may be scheduled while the previous
+    // one finishes (it waits for it in-kernel before reading its results)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c.grid);
+    cfg.blockDim = dim3(c.consumers + 32);
+    cfg.dynamicSmemBytes = c.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <int MODE, int MAXM>
@@ -765,7 +781,7 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
     p.vec_bytes = p.resident ? (uint32_t)xres
                              : (mode == 0 ? (uint32_t)c.maxm * p.K * 4u
                                           : (uint32_t)c.maxm * p.U * kDigitRecBytes);
-    const uint32_t nvec = p.resident ? 1 : 2;
+    const uint32_t nvec = p.resident ? 1 : kVecBufs;
     p.off_vec = align_up(p.off_red + red_bytes, 128);
     p.off_stage = align_up(p.off_vec + nvec * p.vec_bytes, 128);
     p.sc_area = align_up((uint32_t)p.SR * (p.K / 32) + 32, 16);

@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     __shared__ double part[8][RB * kSmallT];
     __shared__ int is_last;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_launch_dependents();   // the expert kernels may be scheduled now; they wait for us
     const int e0 = blockIdx.x * RB;
     const int H4 = p.H / 4;
     const XT* x = reinterpret_cast<const XT*>(p.x);
