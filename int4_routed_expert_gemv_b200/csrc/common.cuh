@@ -80,16 +80,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait until the barrier phase with the given parity has completed.  Gives up after
-// kWaitBudgetNs, records DEV_TIMEOUT and returns false.
+// Wait until the barrier phase with the given parity has completed.  Gives up after about
+// kWaitBudgetCycles SM clock cycles (about 2 s at the B200's clocks), records DEV_TIMEOUT
+// and returns false.  The budget is kept with the SM-local cycle counter: reading it costs
+// a cycle, where the global nanosecond timer is a slow, coarse register.
+constexpr long long kWaitBudgetCycles = 4000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
                                           uint32_t site)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+    const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitBudgetNs) {
+        if (clock64() - t0 > kWaitBudgetCycles) {
             set_flag(status, DEV_TIMEOUT);
             atomicExch(status + 3, site);   // WsHeader::timeout_site
             return false;

@@ -53,6 +53,7 @@ struct Task {
     int tok0;     // first token of the segment in this task
     int ntok;     // tokens in this task (<= Nmax)
     int rb;       // 128-row block of the weight matrix
+    int expert;   // the segment's expert, -1 for the shared expert
 };
 
 struct GemmParams {
@@ -324,45 +325,64 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         // ---------------------------------- dequantisers ------------------------------
         const int r = (tid - 128) >> 1;        // weight row within the 128-row tile
         const int half = (tid - 128) & 1;      // 16-byte chunks 4*half .. 4*half+3 of the row
+        const uint64_t IH = (uint64_t)p.I * p.H;
+        // this thread's row of fp16 scales for a task: K / 64 consecutive values, read 8 at a
+        // time (16 bytes: the scales of 8 stages) one block ahead, across task boundaries
+        auto scale_row = [&](const Task& tk, int mt) {
+            const uint8_t* blob = tk.expert < 0 ? p.shared : p.experts + (uint64_t)tk.expert * p.stride;
+            const uint64_t soff = phase == 0 ? (3 * IH / 2 + (uint64_t)mt * (IH / 32)) : (3 * IH / 2 + 2 * (IH / 32));
+            return reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(blob + soff) +
+                                                  (size_t)(tk.rb * kRows + r) * (K / 64));
+        };
         uint32_t it = 0;
-        for (int t = blockIdx.x; t < ntasks; t += gridDim.x) {
-            const Task tk = p.tasks[t];
-            const SegView sv = seg_view(p, tk.seg);
-            const uint8_t* blob = sv.expert < 0 ? p.shared : p.experts + (uint64_t)sv.expert * p.stride;
-            const uint64_t IH = (uint64_t)p.I * p.H;
-            // scale rows of this thread's weight row
-            const uint16_t* srow[2];
-            for (int mt = 0; mt < nmat; mt++) {
-                const uint64_t soff = phase == 0 ? (3 * IH / 2 + (uint64_t)mt * (IH / 32))
-                                                 : (3 * IH / 2 + 2 * (IH / 32));
-                srow[mt] = reinterpret_cast<const uint16_t*>(blob + soff) +
-                           (size_t)(tk.rb * kRows + r) * (K / 64);
-            }
-            for (int kc = 0; kc < kchunks; kc++, it++) {
-                const int s = it % kStages;
-                if (!dead && !mbar_wait(&full_in[s], (it / kStages) & 1, p.status, kWaitSite + 3))
-                    dead = true;
-                uint8_t* st = stage_ptr(s);
+        uint4 nb[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        int t = blockIdx.x;
+        Task tk{};
+        if (t < ntasks) {
+            tk = p.tasks[t];
+            for (int mt = 0; mt < nmat; mt++) nb[mt] = __ldg(scale_row(tk, mt));
+        }
+        for (; t < ntasks; t += gridDim.x) {
+            const int tn = t + gridDim.x;
+            const Task tkn = tn < ntasks ? p.tasks[tn] : tk;       // issued early, used last
+            for (int kb = 0; kb < kchunks; kb += 8) {
+                const uint4 cb[2] = {nb[0], nb[1]};
                 for (int mt = 0; mt < nmat; mt++) {
-                    const float sc = __half2float(__ushort_as_half(__ldg(srow[mt] + kc)));
-                    const uint64_t sp = pk2f(sc, sc);
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(st + nmat * a_bytes + b_bytes +
-                                                                     mt * raw_bytes + r * 32 + half * 16);
-                    const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
-                    uint8_t* arow = st + mt * a_bytes + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; c4++) {     // 16-byte chunk c = columns 8c .. 8c+7
-                        const int c = 4 * half + c4;
-                        uint32_t o[4];
-                        dq8_bf16(words[c4], sp, o);
-                        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
+                    if (kb + 8 < kchunks) nb[mt] = __ldg(scale_row(tk, mt) + (kb + 8) / 8);
+                    else if (tn < ntasks) nb[mt] = __ldg(scale_row(tkn, mt));
                 }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[s]);
+#pragma unroll
+                for (int j = 0; j < 8; j++, it++) {
+                    const int s = it % kStages;
+                    if (!dead && !mbar_wait(&full_in[s], (it / kStages) & 1, p.status, kWaitSite + 3))
+                        dead = true;
+                    uint8_t* st = stage_ptr(s);
+#pragma unroll
+                    for (int mt = 0; mt < 2; mt++) {
+                        if (mt >= nmat) break;
+                        const uint32_t cw[4] = {cb[mt].x, cb[mt].y, cb[mt].z, cb[mt].w};
+                        const uint32_t w2 = cw[j >> 1];
+                        const float sc = __half2float(__ushort_as_half((unsigned short)((j & 1) ? (w2 >> 16) : (w2 & 0xFFFFu))));
+                        const uint64_t sp = pk2f(sc, sc);
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(st + nmat * a_bytes + b_bytes +
+                                                                         mt * raw_bytes + r * 32 + half * 16);
+                        const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
+                        uint8_t* arow = st + mt * a_bytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; c4++) {     // 16-byte chunk c = columns 8c .. 8c+7
+                            const int c = 4 * half + c4;
+                            uint32_t o[4];
+                            dq8_bf16(words[c4], sp, o);
+                            *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
+                                make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&a_full[s]);
+                }
             }
+            tk = tkn;
         }
     } else if (warp == 13) {
         // ---------------------------------- MMA issuer --------------------------------
@@ -498,6 +518,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* __rest
 // that share a token tile run close together.  One CTA of 1024 threads: thread s counts the
 // tasks of segment s, a block-wide exclusive scan places them, thread s writes them.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* n_union, const int32_t* offsets,
+                                                    const int32_t* union_ids,
                                                     int T, int k, int n_shared, int I, int H,
                                                     Task* tasks0, int32_t* ntasks0, Task* tasks1,
                                                     int32_t* ntasks1)
@@ -538,10 +559,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* n_union, cons
         p0 += x0 - c0;
         p1 += x1 - c1;
         if (s < nseg) {
+            const int ex = (n_shared && s == 0) ? -1 : union_ids[s - n_shared];
             for (int t0 = 0; t0 < cnt; t0 += kNmax0)
-                for (int rb = 0; rb < rb0; rb++) tasks0[p0++] = Task{s, t0, min(kNmax0, cnt - t0), rb};
+                for (int rb = 0; rb < rb0; rb++) tasks0[p0++] = Task{s, t0, min(kNmax0, cnt - t0), rb, ex};
             for (int t0 = 0; t0 < cnt; t0 += kNmax1)
-                for (int rb = 0; rb < rb1; rb++) tasks1[p1++] = Task{s, t0, min(kNmax1, cnt - t0), rb};
+                for (int rb = 0; rb < rb1; rb++) tasks1[p1++] = Task{s, t0, min(kNmax1, cnt - t0), rb, ex};
         }
         base0 += tot0;
         base1 += tot1;
@@ -701,7 +723,7 @@ cudaError_t gemm_forward(const GemmArgs& a, cudaStream_t s)
                                                 a.residual, a.y);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    plan_kernel<<<1, 1024, 0, s>>>(a.n_union, a.offsets, a.T, a.k, a.n_shared, a.I, a.H, tasks0, counts,
+    plan_kernel<<<1, 1024, 0, s>>>(a.n_union, a.offsets, a.union_ids, a.T, a.k, a.n_shared, a.I, a.H, tasks0, counts,
                                  tasks1, counts + 1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
