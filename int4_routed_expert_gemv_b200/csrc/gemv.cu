@@ -750,10 +750,14 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
     p.N = mode == 0 ? p.I : p.H;
     p.U = p.K / 32;
     if (p.K % 64 || p.U < 2) return false;
+    // tokens per chunk: small batches spread over many experts, so most routed segments
+    // hold one token; one-token chunks keep 8 rows per stage (the shared expert's rows are
+    // then re-read per token, from L2).  The down projection of a short intermediate
+    // dimension keeps 4-token chunks: its per-chunk h loads, not its rows, set the pace.
     if (mode == 0)
-        c.maxm = p.T <= 1 ? 1 : (p.T <= 2 ? 2 : (p.T <= 4 ? 4 : 2));
+        c.maxm = p.T <= 8 ? 1 : 2;
     else
-        c.maxm = p.T <= 1 ? 1 : (p.T <= 2 ? 2 : 4);
+        c.maxm = p.T <= 1 ? 1 : (p.T <= 8 && p.I >= 1024 ? 1 : 4);
     c.consumers = consumers_for(c.maxm);
     const int kV = values_for(c.maxm);
     if (p.U >= 32) {
