@@ -29,8 +29,11 @@
  *   weight[r][c] = q[r][c] * scale[r][c / 64].  Blob size 1.59375 * H * I bytes.
  *
  * Arithmetic contracts (selected by the activation dtype, never silently):
- *   COLI_F32  decode GEMV path: weights are applied exactly (q * scale in fp32), all
- *             products and sums in fp32 (routing in fp64), h kept in fp32.
+ *   COLI_F32  decode GEMV path: weights are applied exactly (q * scale); activations
+ *             (x, and h for the down projection) enter as three 8-bit digits per value
+ *             relative to the largest magnitude of each 32-column unit (about 2^-17 of
+ *             that magnitude), each unit's dot product is an exact integer sum, scaled
+ *             and accumulated in fp32 (routing in fp64).
  *   COLI_BF16 prefill path: x is bf16; every dequantised weight is rounded to bf16
  *             (nearest-even), products accumulate in fp32 on the tensor cores, and h
  *             enters the down projection as a pair of bf16 values (hi = bf16(h),
