@@ -479,6 +479,29 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             const int nrw = (int)(r1 - r0);
             for (int rr = tid; rr < nrw; rr += NCONS) {
                 const int r = (int)r0 + rr;
+                if (p.T <= 8) {
+                    // small batches: one register per token, y read and written once per
+                    // flush; the additions keep the chunk order
+                    for (int t = 0; t < p.T; t++) {
+                        float* yp = p.y + (size_t)t * p.H + r;
+                        float v = *yp;
+                        for (int c = 0; c < nch; c++) {
+                            const ChunkMeta& cm = meta[c];
+                            const int rl_ = r - cm.row0;
+                            if (rl_ < 0 || rl_ >= cm.nrows) continue;
+                            const float* pc = part + cm.part_off;
+                            for (int m = 0; m < cm.M; m++) {
+                                if (cm.tok[m] != t) continue;
+                                const float* q = pc + (size_t)(rl_ * MAXM + m) * nwg;
+                                float d = 0.0f;
+                                for (int w2 = 0; w2 < nwg; w2++) d += q[w2];
+                                v = v + cm.wt[m] * d;
+                            }
+                        }
+                        *yp = v;
+                    }
+                    continue;
+                }
                 for (int c = 0; c < nch; c++) {
                     const ChunkMeta& cm = meta[c];
                     const int rl_ = r - cm.row0;

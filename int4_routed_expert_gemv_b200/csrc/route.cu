@@ -57,10 +57,11 @@ __device__ __forceinline__ float key_value(uint64_t key)
     return __uint_as_float(b);
 }
 
-// One warp selects the top-k of one token's logits and writes idx/w.
+// One warp selects the top-k of one token's logits and writes idx/w.  MAXPL keys per lane
+// (E <= 32 * MAXPL).
+template <int MAXPL>
 __device__ void topk_warp(const float* lt, int E, int k, int32_t* idx_t, float* w_t, int lane)
 {
-    constexpr int MAXPL = kMaxExperts / 32;
     uint64_t key[MAXPL];
 #pragma unroll
     for (int i = 0; i < MAXPL; i++) {
@@ -92,40 +93,12 @@ __device__ void topk_warp(const float* lt, int E, int k, int32_t* idx_t, float* 
     }
 }
 
-// Top-k of every token of a small batch by the whole block: thread i ranks pair
-// (t, e) = (i / E, i % E) against all E keys of its token in shared memory (keys are
-// unique, so ranks are a permutation); rank < k gives the slot.  Weights by one warp per
-// token.  smem: T*E keys (8 bytes) + T*k floats.
-__device__ void topk_block(const RouteParams& p, uint8_t* smem)
+__device__ __forceinline__ void topk_warp_any(const float* lt, int E, int k, int32_t* idx_t, float* w_t,
+                                              int lane)
 {
-    uint64_t* skey = reinterpret_cast<uint64_t*>(smem);
-    float* ssel = reinterpret_cast<float*>(skey + (size_t)p.T * p.E);
-    const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5, lane = tid & 31;
-    const int TE = p.T * p.E;
-    for (int i = tid; i < TE; i += nt) {
-        const int t = i / p.E, e = i - t * p.E;
-        skey[i] = topk_key(__ldcg(p.logits + (size_t)t * p.E + e), e);
-    }
-    __syncthreads();
-    for (int i = tid; i < TE; i += nt) {
-        const int t = i / p.E;
-        const uint64_t* kt = skey + (size_t)t * p.E;
-        const uint64_t me = skey[i];
-        int rank = 0;
-#pragma unroll 8
-        for (int e2 = 0; e2 < p.E; e2++) rank += (kt[e2] > me) ? 1 : 0;
-        if (rank < p.k) {
-            p.idx[(size_t)t * p.k + rank] = i - t * p.E;
-            ssel[t * p.k + rank] = key_value(me);
-        }
-    }
-    __syncthreads();
-    for (int t = warp; t < p.T; t += nt / 32) {
-        double ex = 0.0;
-        if (lane < p.k) ex = exp((double)ssel[t * p.k + lane] - (double)ssel[t * p.k]);
-        const double z = dsum_warp(ex);
-        if (lane < p.k) p.w[(size_t)t * p.k + lane] = (float)(ex / z);
-    }
+    if (E <= 256) topk_warp<8>(lt, E, k, idx_t, w_t, lane);
+    else if (E <= 512) topk_warp<16>(lt, E, k, idx_t, w_t, lane);
+    else topk_warp<kMaxExperts / 32>(lt, E, k, idx_t, w_t, lane);
 }
 
 // Small batches: a CTA computes RB router rows for all T (<= kSmallT) tokens; threads
@@ -208,7 +181,10 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    topk_block(p, smem);
+    // one warp per token (T <= kSmallT = 8 warps of this block)
+    for (int t = warp; t < p.T; t += 8)
+        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k, p.w + (size_t)t * p.k,
+                      lane);
     if (p.do_union) {
         __threadfence();
         __syncthreads();
@@ -223,10 +199,10 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     }
 }
 
-// Large batches: 32 tokens x 32 experts per CTA, 32-column slabs converted to double once
+// Large batches, few tiles (small E): 32 tokens x 32 experts per CTA, 32-column slabs converted to double once
 // when staged in shared memory; each thread accumulates 2 x 2 logits in double.
 template <typename XT>
-__global__ void __launch_bounds__(256) router_tiled_kernel(const __grid_constant__ RouteParams p)
+__global__ void __launch_bounds__(256) router_tiled32_kernel(const __grid_constant__ RouteParams p)
 {
     __shared__ __align__(16) double xs[32][34];   // [k][token]
     __shared__ __align__(16) double ws[32][34];   // [k][expert]
@@ -276,13 +252,89 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(const __grid_constant
         }
 }
 
+// Large batches: 64 tokens x 64 experts per CTA, 16-column slabs of x and W_r converted to
+// double once when staged in shared memory (two slabs in flight); each thread accumulates
+// a 4 x 4 block of logits in double, reading 8 doubles per 16 FMAs.
+template <typename XT>
+__global__ void __launch_bounds__(256) router_tiled64_kernel(const __grid_constant__ RouteParams p)
+{
+    constexpr int TM = 64, KS = 16;
+    __shared__ __align__(16) double xs[2][KS][TM + 2];   // [buf][k][token]
+    __shared__ __align__(16) double ws[2][KS][TM + 2];   // [buf][k][expert]
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.y * TM, e0 = blockIdx.x * TM;
+    const int ty = tid / 16, tx = tid % 16;       // 4 tokens x 4 experts per thread
+    const XT* x = reinterpret_cast<const XT*>(p.x);
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) acc[i][j] = 0.0;
+    // staging: thread -> (row = tid / 4, four consecutive k at 4 * (tid % 4))
+    const int row = tid / 4, c4 = tid % 4;
+    auto load = [&](int k0, float4& xv, float4& wv) {
+        xv = make_float4(0.f, 0.f, 0.f, 0.f);
+        wv = xv;
+        if (t0 + row < p.T) xv = load_x4<XT>(x, ((size_t)(t0 + row) * p.H + k0) / 4 + c4);
+        if (e0 + row < p.E)
+            wv = __ldg(reinterpret_cast<const float4*>(p.w_router) + ((size_t)(e0 + row) * p.H + k0) / 4 + c4);
+    };
+    auto stage = [&](int b, const float4& xv, const float4& wv) {
+        xs[b][c4 * 4 + 0][row] = xv.x;
+        xs[b][c4 * 4 + 1][row] = xv.y;
+        xs[b][c4 * 4 + 2][row] = xv.z;
+        xs[b][c4 * 4 + 3][row] = xv.w;
+        ws[b][c4 * 4 + 0][row] = wv.x;
+        ws[b][c4 * 4 + 1][row] = wv.y;
+        ws[b][c4 * 4 + 2][row] = wv.z;
+        ws[b][c4 * 4 + 3][row] = wv.w;
+    };
+    float4 xv, wv;
+    load(0, xv, wv);
+    stage(0, xv, wv);
+    __syncthreads();
+    const int nk = p.H / KS;
+    for (int kt = 0; kt < nk; kt++) {
+        const int b = kt & 1;
+        if (kt + 1 < nk) load((kt + 1) * KS, xv, wv);   // next slab in flight during the FMAs
+#pragma unroll
+        for (int kk = 0; kk < KS; kk++) {
+            const double2 a01 = *reinterpret_cast<const double2*>(&xs[b][kk][ty * 4]);
+            const double2 a23 = *reinterpret_cast<const double2*>(&xs[b][kk][ty * 4 + 2]);
+            const double2 b01 = *reinterpret_cast<const double2*>(&ws[b][kk][tx * 4]);
+            const double2 b23 = *reinterpret_cast<const double2*>(&ws[b][kk][tx * 4 + 2]);
+            const double av[4] = {a01.x, a01.y, a23.x, a23.y};
+            const double bv[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
+        }
+        if (kt + 1 < nk) stage(b ^ 1, xv, wv);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+            if (t < p.T && e < p.E) {
+                double s = acc[i][j];
+                if (p.bias) s += (double)p.bias[e];
+                const float l = (float)s;
+                if (!isfinite(l)) set_flag(p.status, DEV_NONFINITE);
+                p.logits[(size_t)t * p.E + e] = l;
+            }
+        }
+}
+
 __global__ void __launch_bounds__(256) topk_kernel(const __grid_constant__ RouteParams p)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t < p.T)
-        topk_warp(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
-                  p.w + (size_t)t * p.k, lane);
+        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
+                      p.w + (size_t)t * p.k, lane);
 }
 
 __global__ void __launch_bounds__(1024) union_kernel(const __grid_constant__ RouteParams p)
@@ -305,9 +357,7 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
     if (p.T <= kSmallT) {
         constexpr int RB = 2;
         const int grid = (p.E + RB - 1) / RB;
-        const size_t topk_smem = (size_t)p.T * p.E * 8 + (size_t)p.T * p.k * 4;
-        const size_t union_smem = (p.do_union && p.T * p.k > 32) ? union_smem_bytes(p.E, 8) : 0;
-        const size_t smem = topk_smem > union_smem ? topk_smem : union_smem;
+        const size_t smem = (p.do_union && p.T * p.k > 32) ? union_smem_bytes(p.E, 8) : 0;
         auto kern = bf16 ? router_small_kernel<__nv_bfloat16, RB> : router_small_kernel<float, RB>;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -317,11 +367,22 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
         kern<<<grid, 256, smem, s>>>(p);
         return cudaGetLastError();
     }
-    dim3 grid((p.E + 31) / 32, (p.T + 31) / 32);
-    if (bf16)
-        router_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
-    else
-        router_tiled_kernel<float><<<grid, 256, 0, s>>>(p);
+    // 64 x 64 tiles (4 x 4 logits per thread, half the shared-memory reads per FMA) when
+    // they still give about one CTA per SM, else 32 x 32 tiles for more CTAs
+    const long tiles64 = (long)((p.E + 63) / 64) * ((p.T + 63) / 64);
+    if (tiles64 >= 120) {
+        dim3 grid((p.E + 63) / 64, (p.T + 63) / 64);
+        if (bf16)
+            router_tiled64_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+        else
+            router_tiled64_kernel<float><<<grid, 256, 0, s>>>(p);
+    } else {
+        dim3 grid((p.E + 31) / 32, (p.T + 31) / 32);
+        if (bf16)
+            router_tiled32_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+        else
+            router_tiled32_kernel<float><<<grid, 256, 0, s>>>(p);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !p.do_topk) return e;
     topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p);

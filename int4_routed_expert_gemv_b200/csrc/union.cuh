@@ -64,12 +64,20 @@ static __device__ void union_block(int E, int k, int T, const int32_t* __restric
     }
     for (int i = tid; i < nwarps * E; i += nt) wc[i] = 0;
     __syncthreads();
-    for (int a = tid; a < n; a += nt) {
-        const int e = idx[a];
-        if (e < 0 || e >= E)
-            set_flag(status, DEV_BAD_INDEX);
-        else
-            atomicAdd(&count[e], 1);
+    // counts: lanes of a warp holding the same id add once (hot experts would otherwise
+    // serialise on one shared-memory address)
+    for (int base = 0; base < n; base += nt) {
+        const int a = base + tid;
+        int e = -1;
+        if (a < n) {
+            e = idx[a];
+            if (e < 0 || e >= E) {
+                set_flag(status, DEV_BAD_INDEX);
+                e = -1;
+            }
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&count[e], __popc(peers));
     }
     for (int t = tid; t < T; t += nt)
         for (int s = 1; s < k; s++)
