@@ -479,9 +479,9 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             const int nrw = (int)(r1 - r0);
             for (int rr = tid; rr < nrw; rr += NCONS) {
                 const int r = (int)r0 + rr;
-                if (p.T <= 8) {
-                    // small batches: one register per token, y read and written once per
-                    // flush; the additions keep the chunk order
+                if (p.T == 1) {
+                    // one token: y read and written once per flush, the additions in chunk
+                    // order in a register
                     for (int t = 0; t < p.T; t++) {
                         float* yp = p.y + (size_t)t * p.H + r;
                         float v = *yp;
@@ -528,6 +528,11 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     int32_t dcorr[MAXM][3];
     float dfac[MAXM];
     uint32_t it = 0, vit = 0;
+    // resident activations: a slot's digits stay valid while its token is unchanged
+    // (every chunk of a one-token batch uses the same x)
+    int dtok[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; m++) dtok[m] = -1;
 
     for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
         const Seg g = seg_info(p, s);
@@ -577,7 +582,9 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
                         row_in_vec = tok;
                     }
                     if (MODE == 0) {
-                        load_digits(vsrc + (size_t)row_in_vec * K + 32 * j, dg[m], dcorr[m], dfac[m]);
+                        if (MAXM > 1 || !p.resident || dtok[m] != row_in_vec)   // one-token chunks only
+                            load_digits(vsrc + (size_t)row_in_vec * K + 32 * j, dg[m], dcorr[m], dfac[m]);
+                        dtok[m] = p.resident ? row_in_vec : -1;
                     } else {
                         const uint4* rec = reinterpret_cast<const uint4*>(
                             reinterpret_cast<const uint8_t*>(vsrc) +
@@ -602,6 +609,7 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
                         for (int q = 0; q < 8; q++) dg[m][d][q] = 0u;
                     }
                     dfac[m] = 0.0f;
+                    dtok[m] = -1;
                 }
             }
             if (!p.resident) {
