@@ -62,6 +62,21 @@ def parse():
 # helpers
 # ------------------------------------------------------------------------------------
 
+def max_over_ranks(values, world, device="cpu"):
+    """Each value's maximum over the ranks (one all-reduce; NCCL with device tensors, gloo
+    with CPU tensors).  Timings of a multi-GPU run are the slowest rank's."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu().tolist()]
+
+
+def job_rate(units_per_rank, world, total_ms):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / (total_ms * 1e-3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -392,10 +407,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms = float(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(K)))
         e2e = (e2e_ms, T * H * 4, T * H * 4)
 
-    times = torch.tensor([total_ms, e2e[0] if e2e else 0.0], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms = float(times[0]), float(times[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e[0] if e2e else 0.0], world, dev)
     if rank != 0:
         return None
 
@@ -431,7 +443,7 @@ def run_ours(args, rank, world, local_rank):
     dom = max((n for n in kernels if n != "rmsnorm"), key=lambda n: kernels[n]["share"])
     traffic = recorded_traffic(dom, wl.name)
     tokens = T * K * world
-    value = tokens / (total_ms * 1e-3)
+    value = job_rate(T * K, world, total_ms)
     launches_per_step = NL * ((1 if T <= 8 else 3) + 2 + (1 if stack else 0))
 
     out = {
@@ -581,10 +593,7 @@ def run_prefill(args, wl, rank, world, dev):
             ev2[i][1].record()
         torch.cuda.synchronize(dev)
         e2e_ms = float(sum(ev2[i][0].elapsed_time(ev2[i][1]) for i in range(K)))
-    times = torch.tensor([total_ms, e2e_ms or 0.0], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms2 = float(times[0]), float(times[1])
+    total_ms, e2e_ms2 = max_over_ranks([total_ms, e2e_ms or 0.0], world, dev)
     if rank != 0:
         return None
     flops = 2.0 * 3.0 * H * I * T * (k + s.n_shared)          # useful: every routed token + shared
@@ -594,7 +603,7 @@ def run_prefill(args, wl, rank, world, dev):
     tokens = T * K * world
     out = {
         "metric": "MoE-layer tokens/s; grouped-GEMM bf16 TFLOP/s as fraction of B200 dense peak (prefill)",
-        "value": round(tokens / (total_ms * 1e-3), 1),
+        "value": round(job_rate(T * K, world, total_ms), 1),
         "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(total_ms / K, 4),
