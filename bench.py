@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--pool", type=int, default=64, help="distinct token batches rotated over")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--api", default="layer", choices=["layer", "calls"],
+                    help="timed step: one coli_moe_layer call per layer, or the separate "
+                         "route_union / gate_up / down calls")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: time budget of the timed oracle steps")
@@ -102,6 +105,7 @@ KERNEL_SOURCES = {
              "int4_routed_expert_gemv_b200/csrc/gemv.cuh",
              "int4_routed_expert_gemv_b200/csrc/common.cuh"],
     "route_union": ["int4_routed_expert_gemv_b200/csrc/route.cu",
+                    "int4_routed_expert_gemv_b200/csrc/select.cuh",
                     "int4_routed_expert_gemv_b200/csrc/union.cuh"],
 }
 
@@ -268,16 +272,29 @@ def run_ours(args, rank, world, local_rank):
         else:
             layer_calls(0, xs[i % R], ev, 0)
 
+    def layer_api(l, x_in):
+        """One layer through the single-call API (routing fused into the expert launches)."""
+        if stack:
+            B.check(B.coli_rmsnorm(H, T, x_in, gamma, 1e-5, n_work), "rmsnorm")
+            act, res, y = n_work, x_in, x_in
+        else:
+            act, res, y = x_in, None, bufs.y
+        B.check(B.coli_moe_layer(dims, layers[l]["weights"], act, T, bufs.idx, bufs.w, None,
+                                 bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign, res, y,
+                                 bufs.ws), "coli_moe_layer")
+
+    one_layer = layer_api if args.api == "layer" else (lambda l, x_in: layer_calls(l, x_in, None, 0))
+
     def step_coarse(i, ev):
-        """The same launches with events only around the whole step (no event nodes between
-        kernels, so consecutive launches keep their programmatic dependency)."""
+        """The step with events only around it (no event nodes between kernels, so
+        consecutive launches keep their programmatic dependency)."""
         ev[0].record()
         if stack:
             x_work.copy_(xs[i % R])
             for l in range(NL):
-                layer_calls(l, x_work, None, 0)
+                one_layer(l, x_work)
         else:
-            layer_calls(0, xs[i % R], None, 0)
+            one_layer(0, xs[i % R])
         ev[1].record()
 
     # union size of every (batch, layer), deterministic, for the byte counts
@@ -465,7 +482,10 @@ def run_ours(args, rank, world, local_rank):
                    "weights": "gs64 int4, fp16 scales", "activations": "fp32",
                    "l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
                    "timing": "CUDA graphs of up to 128 steps; events around each step (the value); "
-                             "per-kernel figures from a second pass with events around each launch",
+                             "per-kernel figures from a second pass with events around each launch "
+                             "(separate route_union / gate_up / down calls)",
+                   "api": ("coli_moe_layer, one call per layer" if args.api == "layer"
+                           else "coli_moe_route_union + coli_moe_gate_up + coli_moe_down"),
                    "token_pool": R, "parallelism": f"replicas x{world}",
                    "mean_union_per_layer": float(nu.mean() / NL)},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gb_s"],

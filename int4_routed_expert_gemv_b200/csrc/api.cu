@@ -377,10 +377,22 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* we
     p.n_union = n_union;
     p.offsets = offsets;
     p.assign = assign;
-    cudaError_t e = route_launch(p, (cudaStream_t)stream);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = route_launch(p, s);
     if (e != cudaSuccess) return COLI_ECUDA;
-    return coli_moe_forward(dims, weights, x, dtype, T, idx, w, union_ids, n_union, offsets, assign,
-                            residual, y, ws, ws_bytes, stream);
+    if (dtype == COLI_BF16)
+        return coli_moe_forward(dims, weights, x, dtype, T, idx, w, union_ids, n_union, offsets,
+                                assign, residual, y, ws, ws_bytes, stream);
+    // x was complete before the router launch began (an ordinary stream-ordered launch), so
+    // the gate/up launch may stage it while the router still runs
+    GemvParams g = gemv_params(dims, weights, reinterpret_cast<const float*>(x), T, w, union_ids,
+                               n_union, offsets, assign, residual, y, ws);
+    g.x_early = 1;
+    coli_status r = run_gemv(0, g, s);
+    if (r != COLI_OK) return r;
+    GemvParams q = gemv_params(dims, weights, nullptr, T, w, union_ids, n_union, offsets, assign,
+                               residual, y, ws);
+    return run_gemv(1, q, s);
 }
 
 coli_status coli_rmsnorm(int32_t hidden, int32_t T, const float* x, const float* gamma, double eps,

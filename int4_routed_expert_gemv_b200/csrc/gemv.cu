@@ -16,15 +16,17 @@
 //     completing on mbarriers; activations (x, or h for the down projection) arrive the
 //     same way into vector buffers;
 //   * consumer thread (rho, j) owns 16-byte column unit j (32 int4 weights = half a
-//     group) of every row rho, rho+rl, ... of a stage, keeps the matching 32 activations
-//     of each token in registers, and dequantises in registers: a nibble is placed into
-//     the mantissa of a float with a fixed exponent (one LOP3), the exponent's offset is
-//     removed by a packed f32x2 add (exact), and f32x2 FMAs accumulate q*x; the partial
-//     is scaled by the group scale, so every product and scale is exact before rounding;
+//     group) of every row rho, rho+rl, ... of a stage.  The unit's activations are held in
+//     registers as three int8 digit planes with one scale factor (load_digits for x; the
+//     gate/up launch writes h in the same form), so one unit's dot product is 24 dp4a on
+//     the offset-binary nibble bytes, exact in int32, then one scaling by digit factor
+//     times group scale;
 //   * per stage, the partials of the 8 values a thread holds are reduced across the
 //     lanes of a row with a transposing butterfly (each shuffle halves the values a lane
 //     keeps), then across warps through shared memory; finalizer threads apply SwiGLU
 //     (mode 0) or the routing weight and the fixed-order combine into y (mode 1).
+// In the decode layer call x was complete before the router launch began, so the gate/up
+// launch stages it and forms token 0's digits while the router still runs.
 // Every wait on an mbarrier is bounded; a timeout marks the workspace status word and
 // the CTA runs to completion without further waiting, so no launch can hang.
 #include "common.cuh"
@@ -33,7 +35,6 @@
 namespace coli {
 namespace {
 
-constexpr int kBarFull = 0;      // mbarrier slots in shared memory
 constexpr int kMaxStages = 16;
 constexpr int kMaxChunks = 64;      // pending chunks per flush
 constexpr int kVecBufs = 4;         // activation (x or h digit record) buffers when not resident
@@ -83,50 +84,52 @@ __device__ __forceinline__ int rint_small(float v)
 __device__ __forceinline__ void load_digits(const float* src, uint32_t (&dg)[3][8],
                                             int32_t (&corr)[3], float& fac)
 {
-    float xv[32];
     const float4* s4 = reinterpret_cast<const float4*>(src);
+    float mx = 0.0f;
 #pragma unroll
     for (int q4 = 0; q4 < 8; q4++) {
         const float4 v = s4[q4];
-        xv[4 * q4] = v.x;
-        xv[4 * q4 + 1] = v.y;
-        xv[4 * q4 + 2] = v.z;
-        xv[4 * q4 + 3] = v.w;
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
-    float mx = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 32; c++) mx = fmaxf(mx, fabsf(xv[c]));
     const float inv = mx > 0.0f ? 126.0f / mx : 0.0f;
     fac = mx * (1.0f / (126.0f * 65536.0f));
+    int32_t sum[3] = {0, 0, 0};
 #pragma unroll
-    for (int d = 0; d < 3; d++) {
-        corr[d] = 0;
+    for (int d = 0; d < 3; d++)
 #pragma unroll
         for (int q = 0; q < 8; q++) dg[d][q] = 0u;
+    // byte b of every packed word per pass (a rolled loop keeps the code short): slot s
+    // holds column 8 (s / 2) + 2 b + (s % 2); each pass shifts the earlier bytes down
+#pragma unroll 1
+    for (int b = 0; b < 4; b++) {
+        float2 xv[4];
+#pragma unroll
+        for (int w = 0; w < 4; w++) xv[w] = *reinterpret_cast<const float2*>(src + 8 * w + 2 * b);
+#pragma unroll
+        for (int sl = 0; sl < 8; sl++) {
+            const float xc = (sl & 1) ? xv[sl >> 1].y : xv[sl >> 1].x;
+            const float X = fminf(fmaxf(xc * inv, -126.0f), 126.0f);
+            float a, bq;
+            const int ai = floor_small(X, a);
+            // X - a can round up to exactly 1.0f when X is a tiny negative number; the
+            // second digit then saturates at 255 and the third absorbs the remainder
+            const float r1 = (X - a) * 256.0f;
+            int bi = floor_small(r1, bq);
+            if (bi > 255) {
+                bi = 255;
+                bq = 255.0f;
+            }
+            const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
+            dg[0][sl] = (dg[0][sl] >> 8) | ((uint32_t)ai << 24);
+            dg[1][sl] = (dg[1][sl] >> 8) | ((uint32_t)bi << 24);
+            dg[2][sl] = (dg[2][sl] >> 8) | ((uint32_t)ci << 24);
+            sum[0] += ai;
+            sum[1] += bi;
+            sum[2] += ci;
+        }
     }
 #pragma unroll
-    for (int c = 0; c < 32; c++) {
-        const float X = fminf(fmaxf(xv[c] * inv, -126.0f), 126.0f);
-        float a, bq;
-        const int ai = floor_small(X, a);
-        // X - a can round up to exactly 1.0f when X is a tiny negative number; the second
-        // digit then saturates at 255 and the third absorbs the remainder
-        const float r1 = (X - a) * 256.0f;
-        int bi = floor_small(r1, bq);
-        if (bi > 255) {
-            bi = 255;
-            bq = 255.0f;
-        }
-        const int ci = min(rint_small((r1 - bq) * 256.0f), 255);
-        const int di[3] = {ai, bi, ci};
-        const int wi = c >> 3, k = c & 7;
-        const int slot = 2 * wi + (k & 1), byte = k >> 1;
-#pragma unroll
-        for (int d = 0; d < 3; d++) {
-            dg[d][slot] |= ((uint32_t)di[d] & 0xFFu) << (8 * byte);
-            corr[d] -= 8 * di[d];
-        }
-    }
+    for (int d = 0; d < 3; d++) corr[d] = -8 * sum[d];
 }
 
 // A warp turns 32 consecutive activations (lane l holds column l) into one digit record
@@ -331,103 +334,134 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
         fence_barrier_init();
     }
     __syncthreads();
-    // everything above overlaps the previous kernel; routing, activations and h are read
-    // only after it has completed
+
+    // consumer geometry: thread (rho, j) owns column unit j of rows rho, rho + rl, ...
+    const int U = p.U;
+    const int rho = tid / U;
+    const int j = tid - rho * U;
+    const bool active = tid < NCONS && rho < p.rl;
+    bool dead = false;
+    // activations of this thread's 32-column unit as three int8 digits per column,
+    // packed in the byte order of the offset-binary nibble words (see load_digits)
+    uint32_t dg[MAXM][3][8];
+    int32_t dcorr[MAXM][3];
+    float dfac[MAXM];
+    // resident activations: a slot's digits stay valid while its token is unchanged
+    // (every chunk of a one-token batch uses the same x)
+    int dtok[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; m++) dtok[m] = -1;
+
+    // Everything above overlaps the preceding launch.  Routing, h and (unless x_early)
+    // x are read only after it has completed.  An early x is staged now and token 0's
+    // digits are formed while the preceding launch still runs.
+    const bool early_x = MODE == 0 && p.x_early && p.resident;
+    if (early_x) {
+        if (tid == NCONS) {
+            const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
+            mbar_arrive_expect_tx(&vfull[0], bytes);
+            bulk_g2s(vec, p.x, bytes, &vfull[0]);
+        }
+        if (MAXM == 1 && active) {
+            if (!mbar_wait(&vfull[0], 0, p.status, 20)) {
+                dead = true;
+            } else {
+                load_digits(reinterpret_cast<const float*>(vec) + 32 * j, dg[0], dcorr[0], dfac[0]);
+                dtok[0] = 0;
+            }
+        }
+    }
     pdl_wait();
     const int nu = *p.n_union;
     const int nseg = p.n_shared + nu;
 
     if (warp == NCONS / 32) {
         // ------------------------------- producer ------------------------------------
-        if (lane != 0) return;
-        const uint64_t pol = policy_evict_first();
-        bool dead = false;
-        uint32_t it = 0, vit = 0;
-        if (p.resident) {
-            const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
-            mbar_arrive_expect_tx(&vfull[0], bytes);
-            bulk_g2s(vec, p.x, bytes, &vfull[0]);
-        }
-        for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
-            const Seg g = seg_info(p, s);
-            for (int c0 = 0; c0 < g.count; c0 += MAXM) {
-                const int M = min(MAXM, g.count - c0);
-                if (!p.resident) {
-                    const int b = vit % kVecBufs;
-                    if (!dead && !mbar_wait(&vempty[b], ((vit / kVecBufs) & 1) ^ 1, p.status, 11))
-                        dead = true;
-                    if (!dead) {
-                        uint8_t* dst = vec + b * p.vec_bytes;
-                        const uint32_t rowb = (uint32_t)K * 4u;
-                        mbar_arrive_expect_tx(&vfull[b], MODE == 0 ? rowb * M
-                                                                   : (uint32_t)(p.U * kDigitRecBytes) * M);
-                        if (MODE == 0) {
-                            for (int m = 0; m < M; m++) {
-                                int tok;
-                                float wt;
-                                seg_token(p, g, c0 + m, tok, wt);
-                                bulk_g2s(dst + m * rowb, p.x + (size_t)tok * p.H, rowb, &vfull[b]);
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            bool dead = false;
+            uint32_t it = 0, vit = 0;
+            if (p.resident && !early_x) {
+                const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
+                mbar_arrive_expect_tx(&vfull[0], bytes);
+                bulk_g2s(vec, p.x, bytes, &vfull[0]);
+            }
+            for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
+                const Seg g = seg_info(p, s);
+                for (int c0 = 0; c0 < g.count; c0 += MAXM) {
+                    const int M = min(MAXM, g.count - c0);
+                    if (!p.resident) {
+                        const int b = vit % kVecBufs;
+                        if (!dead && !mbar_wait(&vempty[b], ((vit / kVecBufs) & 1) ^ 1, p.status, 11))
+                            dead = true;
+                        if (!dead) {
+                            uint8_t* dst = vec + b * p.vec_bytes;
+                            const uint32_t rowb = (uint32_t)K * 4u;
+                            mbar_arrive_expect_tx(&vfull[b], MODE == 0 ? rowb * M
+                                                                       : (uint32_t)(p.U * kDigitRecBytes) * M);
+                            if (MODE == 0) {
+                                for (int m = 0; m < M; m++) {
+                                    int tok;
+                                    float wt;
+                                    seg_token(p, g, c0 + m, tok, wt);
+                                    bulk_g2s(dst + m * rowb, p.x + (size_t)tok * p.H, rowb, &vfull[b]);
+                                }
+                            } else {
+                                bulk_g2s(dst, p.hd + (size_t)(g.base + c0) * p.U * kDigitRecBytes,
+                                         (uint32_t)(p.U * kDigitRecBytes) * M, &vfull[b]);
                             }
-                        } else {
-                            bulk_g2s(dst, p.hd + (size_t)(g.base + c0) * p.U * kDigitRecBytes,
-                                     (uint32_t)(p.U * kDigitRecBytes) * M, &vfull[b]);
                         }
+                        vit++;
                     }
-                    vit++;
-                }
-                for (int r = 0; r < nrows; r += p.SR) {
-                    const int nr = min(p.SR, nrows - r);
-                    const int row = row0 + r;
-                    const int st = it % p.NS;
-                    if (!dead && !mbar_wait(&empty[st], ((it / p.NS) & 1) ^ 1, p.status, 12))
-                        dead = true;
-                    if (!dead) {
-                        uint8_t* sbase = stages + (size_t)st * p.stage_bytes;
-                        const uint32_t qb = (uint32_t)nr * (uint32_t)(K / 2);
-                        const uint64_t s0 = (uint64_t)row * (K / 32);
-                        const uint64_t a0 = s0 & ~15ull;
-                        const uint64_t a1 = (s0 + (uint64_t)nr * (K / 32) + 15) & ~15ull;
-                        const uint32_t sb = (uint32_t)(a1 - a0);
-                        mbar_arrive_expect_tx(&full[st], NMAT * (qb + sb));
-#pragma unroll
-                        for (int mt = 0; mt < NMAT; mt++) {
-                            bulk_g2s_hint(sbase + (size_t)mt * p.SR * (K / 2),
-                                          g.blob + p.q_off[mt] + (uint64_t)row * (K / 2), qb,
-                                          &full[st], pol);
-                            bulk_g2s_hint(sbase + p.stage_sc_off + mt * p.sc_area,
-                                          g.blob + p.s_off[mt] + a0, sb, &full[st], pol);
+                    for (int r = 0; r < nrows; r += p.SR) {
+                        const int nr = min(p.SR, nrows - r);
+                        const int row = row0 + r;
+                        const int st = it % p.NS;
+                        if (!dead && !mbar_wait(&empty[st], ((it / p.NS) & 1) ^ 1, p.status, 12))
+                            dead = true;
+                        if (!dead) {
+                            uint8_t* sbase = stages + (size_t)st * p.stage_bytes;
+                            const uint32_t qb = (uint32_t)nr * (uint32_t)(K / 2);
+                            const uint64_t s0 = (uint64_t)row * (K / 32);
+                            const uint64_t a0 = s0 & ~15ull;
+                            const uint64_t a1 = (s0 + (uint64_t)nr * (K / 32) + 15) & ~15ull;
+                            const uint32_t sb = (uint32_t)(a1 - a0);
+                            mbar_arrive_expect_tx(&full[st], NMAT * (qb + sb));
+    #pragma unroll
+                            for (int mt = 0; mt < NMAT; mt++) {
+                                bulk_g2s_hint(sbase + (size_t)mt * p.SR * (K / 2),
+                                              g.blob + p.q_off[mt] + (uint64_t)row * (K / 2), qb,
+                                              &full[st], pol);
+                                bulk_g2s_hint(sbase + p.stage_sc_off + mt * p.sc_area,
+                                              g.blob + p.s_off[mt] + a0, sb, &full[st], pol);
+                            }
                         }
+                        it++;
                     }
-                    it++;
                 }
+            });
+            // drain: every issued copy has landed before the CTA may exit
+            const uint32_t n_issued = it < (uint32_t)p.NS ? it : (uint32_t)p.NS;
+            for (uint32_t q = 0; q < n_issued; q++) {
+                const uint32_t last = it - 1 - q;   // most recent use of slot last % NS
+                mbar_wait(&full[last % p.NS], (last / p.NS) & 1, p.status, 13);
             }
-        });
-        // drain: every issued copy has landed before the CTA may exit
-        const uint32_t n_issued = it < (uint32_t)p.NS ? it : (uint32_t)p.NS;
-        for (uint32_t q = 0; q < n_issued; q++) {
-            const uint32_t last = it - 1 - q;   // most recent use of slot last % NS
-            mbar_wait(&full[last % p.NS], (last / p.NS) & 1, p.status, 13);
-        }
-        if (!p.resident) {
-            for (uint32_t q = 0; q < (vit < (uint32_t)kVecBufs ? vit : (uint32_t)kVecBufs); q++) {
-                const uint32_t last = vit - 1 - q;
-                mbar_wait(&vfull[last % kVecBufs], (last / kVecBufs) & 1, p.status, 14);
+            if (!p.resident) {
+                for (uint32_t q = 0; q < (vit < (uint32_t)kVecBufs ? vit : (uint32_t)kVecBufs); q++) {
+                    const uint32_t last = vit - 1 - q;
+                    mbar_wait(&vfull[last % kVecBufs], (last / kVecBufs) & 1, p.status, 14);
+                }
+            } else {
+                mbar_wait(&vfull[0], 0, p.status, 15);
             }
-        } else {
-            mbar_wait(&vfull[0], 0, p.status, 15);
         }
         return;
     }
 
     // --------------------------------- consumers ---------------------------------------
-    const int U = p.U;
-    const int rho = tid / U;
-    const int j = tid - rho * U;
-    const bool active = rho < p.rl;
     const int nwg = (U >= 32) ? (U >> 5) : 1;
     const int wg = (U >= 32) ? (j >> 5) : 0;
     const int lane_l = lane & (L - 1);
-    bool dead = false;
     float* part = red;                                   // partial sums of pending chunks
     ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + p.off_meta);
     int nch = 0;                                         // pending chunks (CTA-uniform)
@@ -522,17 +556,7 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
         part_used = 0;
     };
 
-    // activations of this thread's 32-column unit as three int8 digits per column,
-    // packed in the byte order of the offset-binary nibble words (see load_digits)
-    uint32_t dg[MAXM][3][8];
-    int32_t dcorr[MAXM][3];
-    float dfac[MAXM];
     uint32_t it = 0, vit = 0;
-    // resident activations: a slot's digits stay valid while its token is unchanged
-    // (every chunk of a one-token batch uses the same x)
-    int dtok[MAXM];
-#pragma unroll
-    for (int m = 0; m < MAXM; m++) dtok[m] = -1;
 
     for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
         const Seg g = seg_info(p, s);

@@ -45,6 +45,9 @@ struct GemvParams {
     float* y;                 // [T][H] output
     const float* residual;    // [T][H] or null (down: y = residual + MoE)
     uint32_t* status;         // workspace header
+    // x was complete before the preceding launch began (the layer call's router), so the
+    // gate/up launch stages it and forms token 0's digits before waiting for that launch
+    int x_early;
 };
 
 // One 32-column unit of activations in digit form: three planes of 8 packed bytes, the

@@ -13,6 +13,7 @@
 // exp(l_i - l_max) / sum_j exp(l_j - l_max) over the selected logits, in double.
 #include "common.cuh"
 #include "route.cuh"
+#include "select.cuh"
 #include "union.cuh"
 
 namespace coli {
@@ -40,65 +41,6 @@ __device__ __forceinline__ double dsum_warp(double v)
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
-}
-
-// Order-preserving 64-bit key: larger value first, then smaller index.
-__device__ __forceinline__ uint64_t topk_key(float v, int e)
-{
-    uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);   // -0 and +0 compare equal
-    const uint32_t u = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
-}
-
-__device__ __forceinline__ float key_value(uint64_t key)
-{
-    const uint32_t u = (uint32_t)(key >> 32);
-    const uint32_t b = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
-    return __uint_as_float(b);
-}
-
-// One warp selects the top-k of one token's logits and writes idx/w.  MAXPL keys per lane
-// (E <= 32 * MAXPL).
-template <int MAXPL>
-__device__ void topk_warp(const float* lt, int E, int k, int32_t* idx_t, float* w_t, int lane)
-{
-    uint64_t key[MAXPL];
-#pragma unroll
-    for (int i = 0; i < MAXPL; i++) {
-        const int e = lane + 32 * i;
-        key[i] = (e < E) ? topk_key(__ldcg(lt + e), e) : 0ull;
-    }
-    uint64_t mine = 0;   // key of slot `lane` (lanes < k)
-    for (int s = 0; s < k; s++) {
-        uint64_t best = 0;
-#pragma unroll
-        for (int i = 0; i < MAXPL; i++) best = key[i] > best ? key[i] : best;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
-#pragma unroll
-        for (int i = 0; i < MAXPL; i++)
-            if (key[i] == best) key[i] = 0ull;   // keys are unique (index in low bits)
-        if (lane == s) mine = best;
-    }
-    const double lmax = (double)key_value(__shfl_sync(0xffffffffu, mine, 0));
-    double ex = 0.0;
-    if (lane < k) ex = exp((double)key_value(mine) - lmax);
-    const double z = dsum_warp(ex);
-    if (lane < k) {
-        idx_t[lane] = (int32_t)(0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull));
-        w_t[lane] = (float)(ex / z);
-    }
-}
-
-__device__ __forceinline__ void topk_warp_any(const float* lt, int E, int k, int32_t* idx_t, float* w_t,
-                                              int lane)
-{
-    if (E <= 256) topk_warp<8>(lt, E, k, idx_t, w_t, lane);
-    else if (E <= 512) topk_warp<16>(lt, E, k, idx_t, w_t, lane);
-    else topk_warp<kMaxExperts / 32>(lt, E, k, idx_t, w_t, lane);
 }
 
 // Small batches: a CTA computes RB router rows for all T (<= kSmallT) tokens; threads
@@ -181,21 +123,34 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    // one warp per token (T <= kSmallT = 8 warps of this block)
-    for (int t = warp; t < p.T; t += 8)
-        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k, p.w + (size_t)t * p.k,
-                      lane);
-    if (p.do_union) {
+    // one warp per token (T <= kSmallT = 8 warps of this block); a batch of at most 32
+    // assignments passes its selections to the union through shared memory
+    __shared__ int sel[32];
+    const bool small_union = p.do_union && p.T * p.k <= 32;
+    for (int t = warp; t < p.T; t += 8) {
+        int e;
+        float wv;
+        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, lane, e, wv);
+        if (lane < p.k) {
+            p.idx[(size_t)t * p.k + lane] = e;
+            p.w[(size_t)t * p.k + lane] = wv;
+            if (small_union) sel[t * p.k + lane] = e;
+        }
+    }
+    if (!p.do_union) return;
+    if (small_union) {
+        __syncthreads();
+        if (warp == 0) {
+            const int n = p.T * p.k;
+            const int e = lane < n ? sel[lane] : 0;
+            const UnionLane r = union_warp_lanes(p.E, p.k, n, e, lane, p.status);
+            union_store(r, e, n, p.E, lane, p.union_ids, p.n_union, p.offsets, p.assign);
+        }
+    } else {
         __threadfence();
         __syncthreads();
-        if (p.T * p.k <= 32) {
-            if (warp == 0)
-                union_warp_small(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
-                                 p.status, lane);
-        } else {
-            union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
-                        p.status, smem);
-        }
+        union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status,
+                    smem);
     }
 }
 
@@ -332,18 +287,27 @@ __global__ void __launch_bounds__(256) topk_kernel(const __grid_constant__ Route
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
-    if (t < p.T)
-        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, p.idx + (size_t)t * p.k,
-                      p.w + (size_t)t * p.k, lane);
+    if (t < p.T) {
+        int e;
+        float wv;
+        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, lane, e, wv);
+        if (lane < p.k) {
+            p.idx[(size_t)t * p.k + lane] = e;
+            p.w[(size_t)t * p.k + lane] = wv;
+        }
+    }
 }
 
 __global__ void __launch_bounds__(1024) union_kernel(const __grid_constant__ RouteParams p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     if (p.T * p.k <= 32) {
-        if (threadIdx.x < 32)
-            union_warp_small(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign,
-                             p.status, threadIdx.x);
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x, n = p.T * p.k;
+            const int e = lane < n ? p.idx[lane] : 0;
+            const UnionLane r = union_warp_lanes(p.E, p.k, n, e, lane, p.status);
+            union_store(r, e, n, p.E, lane, p.union_ids, p.n_union, p.offsets, p.assign);
+        }
         return;
     }
     union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status, smem);

@@ -132,57 +132,4 @@ static __device__ void union_block(int E, int k, int T, const int32_t* __restric
     }
 }
 
-// Small batches (T*k <= 32): one warp sorts the (expert, position) keys with a bitonic
-// network and reads the union, offsets and assignment lists off the sorted order.  Same
-// outputs as union_block.  Called by all 32 lanes of one warp.
-static __device__ void union_warp_small(int E, int k, int T, const int32_t* __restrict__ idx,
-                                        int32_t* __restrict__ union_ids,
-                                        int32_t* __restrict__ n_union,
-                                        int32_t* __restrict__ offsets,
-                                        int32_t* __restrict__ assign, uint32_t* status, int lane)
-{
-    const int n = T * k;
-    int e = (lane < n) ? idx[lane] : 0;
-    bool valid = lane < n;
-    if (valid && (e < 0 || e >= E)) {
-        set_flag(status, DEV_BAD_INDEX);
-        valid = false;
-    }
-    // repeated id within a token
-    const int t = lane / k, s = lane - t * k;
-    for (int s2 = 0; s2 < k; s2++) {
-        const int src = t * k + s2;
-        const int o = __shfl_sync(0xffffffffu, e, src < 32 ? src : 0);
-        if (lane < n && src < n && s2 != s && o == e) set_flag(status, DEV_BAD_INDEX);
-    }
-    uint32_t key = valid ? (((uint32_t)e << 8) | (uint32_t)lane) : 0xFFFFFFFFu;
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size / 2; stride > 0; stride >>= 1) {
-            const uint32_t other = __shfl_xor_sync(0xffffffffu, key, stride);
-            const bool up = (lane & size) == 0;
-            const bool lower = (lane & stride) == 0;
-            key = (lower == up) ? min(key, other) : max(key, other);
-        }
-    }
-    const bool ok = key != 0xFFFFFFFFu;
-    const int es = (int)(key >> 8), as = (int)(key & 0xFFu);
-    const int eprev = __shfl_up_sync(0xffffffffu, es, 1);
-    const bool first = ok && (lane == 0 || eprev != es);
-    const unsigned ball = __ballot_sync(0xffffffffu, first);
-    const int nu = __popc(ball);
-    const int u = __popc(ball & ((2u << lane) - 1u)) - 1;
-    if (ok) assign[lane] = as;
-    if (first) {
-        union_ids[u] = es;
-        offsets[u] = lane;
-    }
-    for (int q = nu + lane; q <= E; q += 32) {
-        if (q < E) union_ids[q] = -1;
-        offsets[q] = n;
-    }
-    if (lane == 0) *n_union = nu;
-}
-
 }  // namespace coli
