@@ -170,7 +170,11 @@ COLI_API coli_status coli_moe_down(const coli_moe_dims* dims, const coli_moe_wei
 
 /* Whole layer: route (+ union fused into the router's last block for T <= 8) then
  * forward.  idx, w, union_ids, n_union, offsets, assign are written as by the separate
- * calls; logits may be NULL. */
+ * calls; logits may be NULL.  fp32, T <= 8: x is also turned into activation digits in a
+ * launch of its own (held in the workspace), which the router launch overlaps; larger fp32
+ * batches let the gate/up launch read x before the router launch has finished (x is
+ * complete by then: the first launch of the call is stream-ordered after the caller's
+ * earlier work). */
 COLI_API coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* weights,
                            const void* x, coli_dtype dtype, int32_t T, int32_t* idx, float* w,
                            float* logits, int32_t* union_ids, int32_t* n_union, int32_t* offsets,

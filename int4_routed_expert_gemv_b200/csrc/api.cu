@@ -19,7 +19,7 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t logits, h, gemm, total;
+    size_t logits, h, xd, gemm, total;
 };
 
 bool dims_ok(const coli_moe_dims* d)
@@ -41,6 +41,8 @@ WsLayout ws_layout(const coli_moe_dims* d, int64_t T)
     off += (size_t)T * d->n_experts * sizeof(float);
     L.h = off = up(off, kAlign);
     off += (size_t)T * (d->top_k + d->n_shared) * d->inter * sizeof(float);
+    L.xd = off = up(off, kAlign);
+    off += (size_t)T * (d->hidden / 32) * kDigitRecBytes;
     L.gemm = off = up(off, kAlign);
     off += gemm_workspace_bytes(d->hidden, d->inter, d->n_experts, d->top_k, d->n_shared, T);
     L.total = up(off, kAlign);
@@ -378,16 +380,28 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* we
     p.offsets = offsets;
     p.assign = assign;
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = route_launch(p, s);
-    if (e != cudaSuccess) return COLI_ECUDA;
-    if (dtype == COLI_BF16)
+    if (dtype == COLI_BF16) {
+        if (route_launch(p, s) != cudaSuccess) return COLI_ECUDA;
         return coli_moe_forward(dims, weights, x, dtype, T, idx, w, union_ids, n_union, offsets,
                                 assign, residual, y, ws, ws_bytes, stream);
-    // x was complete before the router launch began (an ordinary stream-ordered launch), so
-    // the gate/up launch may stage it while the router still runs
+    }
     GemvParams g = gemv_params(dims, weights, reinterpret_cast<const float*>(x), T, w, union_ids,
                                n_union, offsets, assign, residual, y, ws);
-    g.x_early = 1;
+    if (T <= kSmallT) {
+        // decode batch: x turns into digit records in a launch of its own, which the router
+        // (a programmatic dependent that waits for it before completing) overlaps
+        uint8_t* xd = (uint8_t*)ws + ws_layout(dims, T).xd;
+        if (x_digits_launch(reinterpret_cast<const float*>(x), T, dims->hidden, xd, s) !=
+            cudaSuccess)
+            return COLI_ECUDA;
+        p.pdl = 1;
+        g.xd = xd;
+    } else {
+        // x was complete before the router launch began (an ordinary stream-ordered
+        // launch), so the gate/up launch may stage it while the router still runs
+        g.x_early = 1;
+    }
+    if (route_launch(p, s) != cudaSuccess) return COLI_ECUDA;
     coli_status r = run_gemv(0, g, s);
     if (r != COLI_OK) return r;
     GemvParams q = gemv_params(dims, weights, nullptr, T, w, union_ids, n_union, offsets, assign,

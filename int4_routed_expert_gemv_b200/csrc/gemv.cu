@@ -181,6 +181,20 @@ __device__ __forceinline__ void store_digit_record(float hv, int lane, uint32_t*
     if (lane < kDigitRecWords) rec[lane] = out;
 }
 
+// x [T][H] into digit records, one warp per 32-column unit (same digits as load_digits).
+__global__ void __launch_bounds__(256) x_digits_kernel(const float* __restrict__ x, int T, int H,
+                                                       uint8_t* __restrict__ rec)
+{
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int U = H / 32;
+    const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (u >= T * U) return;
+    const int t = u / U, j = u - t * U;
+    store_digit_record(x[(size_t)t * H + 32 * j + lane], lane,
+                       reinterpret_cast<uint32_t*>(rec + (size_t)u * kDigitRecBytes));
+}
+
 // Transposing butterfly over W*2 lanes: at each level the lane with bit W set keeps the
 // upper half of its values, sends the lower half, and adds what its partner sends.
 template <int CUR, int W>
@@ -249,16 +263,18 @@ __device__ __forceinline__ void seg_token(const GemvParams& p, const Seg& g, int
 }
 
 template <int MODE>
-__device__ __forceinline__ void cta_rows(const GemvParams& p, int nseg, int64_t& r0, int64_t& r1)
+__device__ __forceinline__ void cta_rows(const GemvParams& p, int nseg, int& r0, int& r1)
 {
+    // 32-bit arithmetic: gemv_plan keeps (E + 1) * N * gridDim below 2^32
+    const uint32_t b = blockIdx.x, G = gridDim.x;
     if (MODE == 0) {
         // whole 32-row units, so every unit of h is finished by one CTA
-        const int64_t R = (int64_t)nseg * (p.N / 32);
-        r0 = 32 * (R * blockIdx.x / gridDim.x);
-        r1 = 32 * (R * (blockIdx.x + 1) / gridDim.x);
+        const uint32_t R = (uint32_t)nseg * (uint32_t)(p.N / 32);
+        r0 = (int)(32u * (R * b / G));
+        r1 = (int)(32u * (R * (b + 1) / G));
     } else {
-        r0 = (int64_t)p.N * blockIdx.x / gridDim.x;
-        r1 = (int64_t)p.N * (blockIdx.x + 1) / gridDim.x;
+        r0 = (int)((uint32_t)p.N * b / G);
+        r1 = (int)((uint32_t)p.N * (b + 1) / G);
     }
 }
 
@@ -267,22 +283,20 @@ __device__ __forceinline__ void cta_rows(const GemvParams& p, int nseg, int64_t&
 template <int MODE, class F>
 __device__ __forceinline__ void for_each_piece(const GemvParams& p, int nseg, F&& f)
 {
-    int64_t r0, r1;
+    int r0, r1;
     cta_rows<MODE>(p, nseg, r0, r1);
     if (MODE == 0) {
-        int64_t r = r0;
+        int r = r0;
         while (r < r1) {
-            const int s = (int)(r / p.N);
-            const int64_t end = min(r1, (int64_t)(s + 1) * p.N);
-            for (int64_t q = r; q < end; q += p.PR)
-                f(s, (int)(q - (int64_t)s * p.N), (int)min((int64_t)p.PR, end - q));
+            const int s = (int)((uint32_t)r / (uint32_t)p.N);
+            const int end = min(r1, (s + 1) * p.N);
+            for (int q = r; q < end; q += p.PR) f(s, q - s * p.N, min(p.PR, end - q));
             r = end;
         }
     } else {
         if (r1 > r0)
             for (int s = 0; s < nseg; s++)
-                for (int64_t q = r0; q < r1; q += p.PR)
-                    f(s, (int)q, (int)min((int64_t)p.PR, r1 - q));
+                for (int q = r0; q < r1; q += p.PR) f(s, q, min(p.PR, r1 - q));
     }
 }
 
@@ -355,7 +369,7 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     // Everything above overlaps the preceding launch.  Routing, h and (unless x_early)
     // x are read only after it has completed.  An early x is staged now and token 0's
     // digits are formed while the preceding launch still runs.
-    const bool early_x = MODE == 0 && p.x_early && p.resident;
+    const bool early_x = MODE == 0 && p.x_early && p.resident && !p.xd;
     if (early_x) {
         if (tid == NCONS) {
             const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
@@ -382,9 +396,15 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
             bool dead = false;
             uint32_t it = 0, vit = 0;
             if (p.resident && !early_x) {
-                const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
-                mbar_arrive_expect_tx(&vfull[0], bytes);
-                bulk_g2s(vec, p.x, bytes, &vfull[0]);
+                if (p.xd) {
+                    const uint32_t bytes = (uint32_t)p.T * (uint32_t)(p.U * kDigitRecBytes);
+                    mbar_arrive_expect_tx(&vfull[0], bytes);
+                    bulk_g2s(vec, p.xd, bytes, &vfull[0]);
+                } else {
+                    const uint32_t bytes = (uint32_t)p.T * (uint32_t)p.H * 4u;
+                    mbar_arrive_expect_tx(&vfull[0], bytes);
+                    bulk_g2s(vec, p.x, bytes, &vfull[0]);
+                }
             }
             for_each_piece<MODE>(p, nseg, [&](int s, int row0, int nrows) {
                 const Seg g = seg_info(p, s);
@@ -396,10 +416,17 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
                             dead = true;
                         if (!dead) {
                             uint8_t* dst = vec + b * p.vec_bytes;
-                            const uint32_t rowb = (uint32_t)K * 4u;
-                            mbar_arrive_expect_tx(&vfull[b], MODE == 0 ? rowb * M
-                                                                       : (uint32_t)(p.U * kDigitRecBytes) * M);
-                            if (MODE == 0) {
+                            const uint32_t recb = (uint32_t)(p.U * kDigitRecBytes);
+                            const uint32_t rowb = (MODE == 0 && !p.xd) ? (uint32_t)K * 4u : recb;
+                            mbar_arrive_expect_tx(&vfull[b], rowb * M);
+                            if (MODE == 0 && p.xd) {
+                                for (int m = 0; m < M; m++) {
+                                    int tok;
+                                    float wt;
+                                    seg_token(p, g, c0 + m, tok, wt);
+                                    bulk_g2s(dst + m * rowb, p.xd + (size_t)tok * recb, rowb, &vfull[b]);
+                                }
+                            } else if (MODE == 0) {
                                 for (int m = 0; m < M; m++) {
                                     int tok;
                                     float wt;
@@ -466,7 +493,7 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
     ChunkMeta* meta = reinterpret_cast<ChunkMeta*>(smem + p.off_meta);
     int nch = 0;                                         // pending chunks (CTA-uniform)
     uint32_t part_used = 0;
-    int64_t r0, r1;
+    int r0, r1;
     cta_rows<MODE>(p, nseg, r0, r1);
 
     if (MODE == 1) {
@@ -605,14 +632,15 @@ __global__ void __launch_bounds__(consumers_for(MAXM) + 32, 1)
                         seg_token(p, g, c0 + m, tok, wt);
                         row_in_vec = tok;
                     }
-                    if (MODE == 0) {
+                    if (MODE == 0 && !p.xd) {
                         if (MAXM > 1 || !p.resident || dtok[m] != row_in_vec)   // one-token chunks only
                             load_digits(vsrc + (size_t)row_in_vec * K + 32 * j, dg[m], dcorr[m], dfac[m]);
                         dtok[m] = p.resident ? row_in_vec : -1;
                     } else {
+                        // digit records: x records of the layer call, or h from the gate/up launch
                         const uint4* rec = reinterpret_cast<const uint4*>(
                             reinterpret_cast<const uint8_t*>(vsrc) +
-                            ((size_t)m * p.U + j) * kDigitRecBytes);
+                            ((size_t)row_in_vec * p.U + j) * kDigitRecBytes);
 #pragma unroll
                         for (int d = 0; d < 3; d++) {
                             const uint4 r0v = rec[2 * d], r1v = rec[2 * d + 1];
@@ -805,6 +833,8 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
     p.N = mode == 0 ? p.I : p.H;
     p.U = p.K / 32;
     if (p.K % 64 || p.U < 2) return false;
+    // the kernels split rows with 32-bit products (segments x rows x CTAs)
+    if ((uint64_t)(p.E + 1) * (uint64_t)p.N * (uint64_t)num_sms >= (1ull << 32)) return false;
     // tokens per chunk: small batches spread over many experts, so most routed segments
     // hold one token; one-token chunks keep 8 rows per stage (the shared expert's rows are
     // then re-read per token, from L2).  The down projection of a short intermediate
@@ -837,9 +867,9 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
     const uint32_t red_bytes = p.part_cap * 4u;
     const uint64_t xres = (uint64_t)p.T * p.H * 4ull;
     p.resident = (mode == 0 && xres <= 100u * 1024u) ? 1 : 0;
-    p.vec_bytes = p.resident ? (uint32_t)xres
-                             : (mode == 0 ? (uint32_t)c.maxm * p.K * 4u
-                                          : (uint32_t)c.maxm * p.U * kDigitRecBytes);
+    const bool recs = mode == 1 || p.xd;   // activations arrive as digit records
+    const uint32_t row_bytes = recs ? (uint32_t)p.U * kDigitRecBytes : (uint32_t)p.K * 4u;
+    p.vec_bytes = p.resident ? (uint32_t)p.T * row_bytes : (uint32_t)c.maxm * row_bytes;
     const uint32_t nvec = p.resident ? 1 : kVecBufs;
     p.off_vec = align_up(p.off_red + red_bytes, 128);
     p.off_stage = align_up(p.off_vec + nvec * p.vec_bytes, 128);
@@ -866,6 +896,14 @@ bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_
         c.grid = p.H < num_sms ? p.H : num_sms;
     }
     return true;
+}
+
+cudaError_t x_digits_launch(const float* x, int T, int H, uint8_t* rec, cudaStream_t s)
+{
+    const int units = T * (H / 32);
+    if (units <= 0) return cudaSuccess;
+    x_digits_kernel<<<(units + 7) / 8, 256, 0, s>>>(x, T, H, rec);
+    return cudaGetLastError();
 }
 
 cudaError_t gemv_launch(int mode, const GemvParams& p, const GemvConfig& c, cudaStream_t s)

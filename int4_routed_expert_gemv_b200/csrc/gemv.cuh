@@ -48,6 +48,9 @@ struct GemvParams {
     // x was complete before the preceding launch began (the layer call's router), so the
     // gate/up launch stages it and forms token 0's digits before waiting for that launch
     int x_early;
+    // gate/up: x already in digit-record form ([T][H/32] records of kDigitRecBytes, written
+    // by x_digits_launch before the preceding launch); read instead of x when set
+    const uint8_t* xd;
 };
 
 // One 32-column unit of activations in digit form: three planes of 8 packed bytes, the
@@ -68,5 +71,10 @@ struct GemvConfig {
 // shape is not supported by the GEMV kernels.
 bool gemv_plan(int mode, GemvParams& p, GemvConfig& c, int num_sms, size_t smem_limit);
 cudaError_t gemv_launch(int mode, const GemvParams& p, const GemvConfig& c, cudaStream_t s);
+
+// x [T][H] fp32 -> digit records rec [T][H/32] (one warp per 32-column unit).  The kernel
+// lets the next launch start at once (programmatic dependent launch); that launch must
+// wait for this grid before anything reads rec.
+cudaError_t x_digits_launch(const float* x, int T, int H, uint8_t* rec, cudaStream_t s);
 
 }  // namespace coli

@@ -111,7 +111,10 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
             p.logits[(size_t)t * p.E + e0 + r] = l;
         }
     }
-    if (!p.do_topk) return;
+    if (!p.do_topk) {
+        pdl_wait();
+        return;
+    }
     // ---- last-CTA election: the final arrival sees every logit
     __threadfence();
     __syncthreads();
@@ -123,30 +126,37 @@ __global__ void __launch_bounds__(256) router_small_kernel(const __grid_constant
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    // one warp per token (T <= kSmallT = 8 warps of this block); a batch of at most 32
-    // assignments passes its selections to the union through shared memory
+    pdl_wait();   // a programmatic launch completes only after the kernel it follows
+    // one warp per token (T <= kSmallT = 8 warps of this block) selects; then warp 0 builds
+    // the union of a batch of at most 32 assignments (selections passed through shared
+    // memory) while the other warps compute the routing weights from the selected keys
     __shared__ int sel[32];
+    __shared__ uint32_t selkey[kSmallT * kMaxTopK];
     const bool small_union = p.do_union && p.T * p.k <= 32;
     for (int t = warp; t < p.T; t += 8) {
         int e;
-        float wv;
-        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, lane, e, wv);
+        uint32_t key;
+        topk_warp_any(p.logits + (size_t)t * p.E, p.E, p.k, lane, e, key);
         if (lane < p.k) {
             p.idx[(size_t)t * p.k + lane] = e;
-            p.w[(size_t)t * p.k + lane] = wv;
+            selkey[t * p.k + lane] = key;
             if (small_union) sel[t * p.k + lane] = e;
         }
     }
-    if (!p.do_union) return;
-    if (small_union) {
-        __syncthreads();
-        if (warp == 0) {
-            const int n = p.T * p.k;
-            const int e = lane < n ? sel[lane] : 0;
-            const UnionLane r = union_warp_lanes(p.E, p.k, n, e, lane, p.status);
-            union_store(r, e, n, p.E, lane, p.union_ids, p.n_union, p.offsets, p.assign);
-        }
-    } else {
+    __syncthreads();
+    const int wfirst = small_union ? 1 : 0;
+    if (small_union && warp == 0) {
+        const int n = p.T * p.k;
+        const int e = lane < n ? sel[lane] : 0;
+        const UnionLane r = union_warp_lanes(p.E, p.k, n, e, lane, p.status);
+        union_store(r, e, n, p.E, lane, p.union_ids, p.n_union, p.offsets, p.assign);
+    }
+    for (int t = warp - wfirst; t >= 0 && t < p.T; t += 8 - wfirst) {
+        const uint32_t key = lane < p.k ? selkey[t * p.k + lane] : 0u;
+        const float wv = topk_weight(key, p.k, lane);
+        if (lane < p.k) p.w[(size_t)t * p.k + lane] = wv;
+    }
+    if (p.do_union && !small_union) {
         __threadfence();
         __syncthreads();
         union_block(p.E, p.k, p.T, p.idx, p.union_ids, p.n_union, p.offsets, p.assign, p.status,
@@ -328,8 +338,21 @@ cudaError_t route_launch(const RouteParams& p, cudaStream_t s)
                                                  (int)smem);
             if (e != cudaSuccess) return e;
         }
-        kern<<<grid, 256, smem, s>>>(p);
-        return cudaGetLastError();
+        if (!p.pdl) {
+            kern<<<grid, 256, smem, s>>>(p);
+            return cudaGetLastError();
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, p);
     }
     // 64 x 64 tiles (4 x 4 logits per thread, half the shared-memory reads per FMA) when
     // they still give about one CTA per SM, else 32 x 32 tiles for more CTAs

@@ -28,6 +28,10 @@ struct RouteParams {
     int32_t* assign;          // [T*k]
     WsHeader* hdr;
     uint32_t* status;         // == &hdr->status
+    // batches up to kSmallT: launch as a programmatic dependent of the previous kernel (which
+    // the router does not read); the grid waits for it before completing, so a launch that
+    // waits for the router also sees everything that kernel wrote
+    int pdl;
 };
 
 cudaError_t route_launch(const RouteParams& p, cudaStream_t s);
