@@ -195,3 +195,37 @@ def test_large_activations_tiny_negative_h(scale):
     ref = oracle_layer(L, x)
     assert_route_union_equal(got, ref)
     assert_y_close(got["y"], ref["y"], rel_l2=1e-5)
+
+
+@pytest.mark.parametrize("H,I,E,k,T", [(1024, 512, 64, 4, 1), (1024, 512, 64, 4, 4),
+                                       (1024, 512, 64, 4, 8), (1024, 512, 64, 4, 9),
+                                       (4096, 256, 16, 4, 7), (4096, 256, 16, 4, 8),
+                                       (4096, 256, 16, 4, 12)])
+def test_layer_call_equals_separate_calls(H, I, E, k, T):
+    # coli_moe_layer forms the activation digits in a launch of its own (T <= 8; x kept
+    # whole in shared memory up to 100 KB, else streamed per chunk) or stages x before the
+    # router has finished (larger T); the separate calls form them inside gate/up.  The
+    # digits are the same, so every output must be the same bit for bit, and match the
+    # oracle.
+    shape = synth.LayerShape(H, I, E, k, 1)
+    L = make_device_layer(shape, 40 + T, zipf=True)
+    x = _x(shape, 40 + T, T, 6)
+    xd = torch.from_numpy(x).cuda()
+    got = run_layer(L, xd, T)
+    ref = oracle_layer(L, x)
+    assert_route_union_equal(got, ref)
+    assert_y_close(got["y"], ref["y"])
+    bufs = B.LayerBuffers(L.dims, T)
+    B.check(B.coli_moe_route_union(L.dims, L.w_router, L.bias, xd, T, bufs.idx, bufs.w,
+                                   bufs.logits, bufs.union_ids, bufs.n_union, bufs.offsets,
+                                   bufs.assign, bufs.ws))
+    B.check(B.coli_moe_gate_up(L.dims, L.weights, xd, T, bufs.union_ids, bufs.n_union,
+                               bufs.offsets, bufs.assign, bufs.ws))
+    B.check(B.coli_moe_down(L.dims, L.weights, T, bufs.w, bufs.union_ids, bufs.n_union,
+                            bufs.offsets, bufs.assign, None, bufs.y, bufs.ws))
+    sep = host_outputs(bufs, T, shape)
+    for key in ("idx", "w", "logits", "union_ids", "offsets", "assign", "y"):
+        assert np.array_equal(got[key], sep[key]), key
+    assert got["n_union"] == sep["n_union"]
+    st, bits = B.coli_moe_read_status(bufs.ws)
+    assert st == B.COLI_OK and bits == 0
