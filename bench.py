@@ -461,7 +461,10 @@ def run_ours(args, rank, world, local_rank):
     traffic = recorded_traffic(dom, wl.name)
     tokens = T * K * world
     value = job_rate(T * K, world, total_ms)
-    launches_per_step = NL * ((1 if T <= 8 else 3) + 2 + (1 if stack else 0))
+    # per layer: router (+ top-k and union kernels above 8 tokens), gate/up, down, the
+    # stack's RMSNorm, and the layer call's x digit-record launch for up to 8 tokens
+    launches_per_step = NL * ((1 if T <= 8 else 3) + 2 + (1 if stack else 0)
+                              + (1 if args.api == "layer" and T <= 8 else 0))
 
     out = {
         "metric": METRIC,
