@@ -203,6 +203,27 @@ COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_dims* dims,
                                               const int32_t* assign, const float* residual,
                                               float* y, void* stream);
 
+/* Residual stack of decode layers, every layer resident in device memory:
+ *   for l in 0 .. n_layers-1:  n = RMSNorm_l(x);  x = x + MoE_l(n);   y = x at the end,
+ * with RMSNorm_l(x) = x * gamma[l] / sqrt(mean(x^2) + eps) (double, rounded once to fp32)
+ * and MoE_l the layer of coli_moe_layer (its shared expert included).  The residual stream
+ * stays on the device from layer to layer (colibri README.zh-CN, "工作原理 / 绝不为同一次
+ * 磁盘读取等待两遍", COLI_CUDA_PIPE=2): up to 16 layers run in one launch, the weights
+ * of each layer streaming while the previous layer finishes.
+ *   layers  host array of n_layers weight descriptors (device pointers inside);
+ *   gamma   host array of n_layers device pointers to [H] fp32 RMSNorm weights, or NULL
+ *           for all-ones; an individual NULL entry also means all-ones;
+ *   x, y    [T][H] fp32 device arrays; y may not overlap x;
+ *   idx     [n_layers][T][k] device array receiving every layer's selected experts (the
+ *           fp32 contract's routing), or NULL.
+ * Decode batches only: 1 <= T <= 4; otherwise (or for a shape the fused kernel does not
+ * take) COLI_EUNSUPPORTED.  fp32 activations (the COLI_F32 contract, except that the
+ * activations entering each layer are quantised with one scale per token). */
+COLI_API coli_status coli_moe_stack(const coli_moe_dims* dims, const coli_moe_weights* layers,
+                                    const float* const* gamma, int32_t n_layers, double eps,
+                                    const float* x, int32_t T, int32_t* idx, float* y, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /* RMSNorm: out [T][H] = x * gamma / sqrt(mean(x^2) + eps), computed in double and
  * rounded once to fp32.  out may alias x. */
 COLI_API coli_status coli_rmsnorm(int32_t hidden, int32_t T, const float* x, const float* gamma, double eps,

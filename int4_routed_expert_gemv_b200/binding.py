@@ -25,7 +25,7 @@ DEV_NONFINITE, DEV_BAD_INDEX, DEV_TIMEOUT, DEV_BAD_SHAPE = 1, 2, 4, 8
 EXPORTS = [
     "coli_moe_blob_bytes", "coli_moe_workspace_bytes", "coli_moe_workspace_init",
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
-    "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_rmsnorm",
+    "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_moe_stack", "coli_rmsnorm",
     "coli_moe_forward_noalloc",
     "coli_status_string",
 ]
@@ -76,6 +76,7 @@ def lib():
                 "coli_moe_gate_up": (i32, [D, W, P, i32, P, P, P, P, P, sz, P]),
                 "coli_moe_down": (i32, [D, W, i32, P, P, P, P, P, P, P, P, sz, P]),
                 "coli_moe_layer": (i32, [D, W, P, i32, i32, P, P, P, P, P, P, P, P, P, P, sz, P]),
+                "coli_moe_stack": (i32, [D, W, P, i32, ctypes.c_double, P, i32, P, P, P, sz, P]),
                 "coli_rmsnorm": (i32, [i32, i32, P, P, ctypes.c_double, P, P]),
                 "coli_moe_forward_noalloc": (i32, [D, W, P, i32, P, P, P, P, P, P, P, P]),
                 "coli_status_string": (ctypes.c_char_p, [i32]),
@@ -196,6 +197,19 @@ def coli_moe_forward_noalloc(dims, weights, x, T, w, union_ids, n_union, offsets
     return lib().coli_moe_forward_noalloc(ctypes.byref(dims), ctypes.byref(weights), _p(x), T,
                                           _p(w), _p(union_ids), _p(n_union), _p(offsets),
                                           _p(assign), _p(residual), _p(y), _s(stream))
+
+
+def coli_moe_stack(dims, layers, gammas, eps, x, T, idx, y, ws, stream=None) -> int:
+    """layers: list of Weights (one per layer); gammas: list of [H] device tensors or None
+    (all-ones RMSNorm weights); idx: [L][T][k] int32 device tensor or None."""
+    n = len(layers)
+    arr = (Weights * max(n, 1))(*layers)
+    if gammas is None:
+        garr = None
+    else:
+        garr = (ctypes.c_void_p * max(n, 1))(*[None if g is None else g.data_ptr() for g in gammas])
+    return lib().coli_moe_stack(ctypes.byref(dims), arr, garr, n, float(eps), _p(x), T, _p(idx),
+                                _p(y), _p(ws), ws.numel(), _s(stream))
 
 
 def coli_rmsnorm(hidden, T, x, gamma, eps, out, stream=None) -> int:

@@ -6,6 +6,7 @@
 
 #include "../../include/colimoe.h"
 #include "common.cuh"
+#include "fused.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
 #include "rmsnorm.cuh"
@@ -19,8 +20,10 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t logits, h, xd, gemm, total;
+    size_t cnt, logits, h, xd, rpart, hf, xbuf, xchunk, gemm, total;
 };
+
+constexpr size_t kCntBytes = (size_t)kCntWords * 4;
 
 bool dims_ok(const coli_moe_dims* d)
 {
@@ -37,12 +40,26 @@ WsLayout ws_layout(const coli_moe_dims* d, int64_t T)
 {
     WsLayout L;
     size_t off = sizeof(WsHeader);
+    // the fused decode kernel's counters sit right after the header (cleared with it)
+    L.cnt = off;
+    off += kCntBytes;
     L.logits = off = up(off, kAlign);
     off += (size_t)T * d->n_experts * sizeof(float);
     L.h = off = up(off, kAlign);
     off += (size_t)T * (d->top_k + d->n_shared) * d->inter * sizeof(float);
     L.xd = off = up(off, kAlign);
     off += (size_t)T * (d->hidden / 32) * kDigitRecBytes;
+    // fused decode kernel (batches up to kFusedMaxT): router partial sums, the layer
+    // outputs of a stack launch, and the outputs of stack launches but the last
+    const int64_t Tf = T < kFusedMaxT ? T : kFusedMaxT;
+    L.rpart = off = up(off, kAlign);
+    off += (size_t)Tf * d->n_experts * (d->hidden / 128 > 0 ? d->hidden / 128 : 1) * sizeof(double);
+    L.hf = off = up(off, kAlign);   // SwiGLU activations as (value, epoch) pairs
+    off += (size_t)Tf * (d->top_k + d->n_shared) * d->inter * 8;
+    L.xbuf = off = up(off, kAlign);
+    off += 2 * (size_t)Tf * d->hidden * sizeof(float);
+    L.xchunk = off = up(off, kAlign);
+    off += 2 * (size_t)Tf * d->hidden * sizeof(float);
     L.gemm = off = up(off, kAlign);
     off += gemm_workspace_bytes(d->hidden, d->inter, d->n_experts, d->top_k, d->n_shared, T);
     L.total = up(off, kAlign);
@@ -146,6 +163,44 @@ GemvParams gemv_params(const coli_moe_dims* d, const coli_moe_weights* wt, const
     return p;
 }
 
+// Fused decode kernel set-up for a batch of T tokens through L layers; false if the shape
+// or batch is outside what the kernel handles (the caller then takes the separate kernels).
+bool fused_setup(FusedParams& f, const coli_moe_dims* d, int32_t T, int L, void* ws)
+{
+    memset(&f, 0, sizeof(f));
+    f.H = d->hidden;
+    f.I = d->inter;
+    f.E = d->n_experts;
+    f.k = d->top_k;
+    f.n_shared = d->n_shared;
+    f.T = T;
+    f.L = L;
+    f.norm = L > 1;
+    DevInfo di;
+    if (!dev_info(di)) return false;
+    if (!fused_plan(f, di.sms, di.smem_optin)) return false;
+    const WsLayout W = ws_layout(d, T);
+    uint8_t* base = (uint8_t*)ws;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    f.status = &hdr->status;
+    f.gen = &hdr->launch_gen;
+    f.cnt = reinterpret_cast<uint32_t*>(base + W.cnt);
+    f.rpart = reinterpret_cast<double*>(base + W.rpart);
+    f.h = reinterpret_cast<uint2*>(base + W.hf);
+    f.xbuf = reinterpret_cast<float*>(base + W.xbuf);
+    return true;
+}
+
+void fused_layer_ptrs(FusedLayer& l, const coli_moe_weights* w, const float* gamma)
+{
+    l.w_router = w->w_router;
+    l.bias = w->router_bias;
+    l.experts = w->experts;
+    l.shared = w->shared;
+    l.gamma = gamma;
+    l.stride = w->expert_stride;
+}
+
 coli_status run_gemv(int mode, GemvParams& p, cudaStream_t s)
 {
     DevInfo di;
@@ -192,7 +247,8 @@ size_t coli_moe_workspace_bytes(const coli_moe_dims* dims, int32_t T_max)
 coli_status coli_moe_workspace_init(void* ws, size_t ws_bytes, void* stream)
 {
     if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return COLI_EINVAL;
-    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream));
+    const size_t n = ws_bytes < sizeof(WsHeader) + kCntBytes ? ws_bytes : sizeof(WsHeader) + kCntBytes;
+    return cuda_status(cudaMemsetAsync(ws, 0, n, (cudaStream_t)stream));
 }
 
 coli_status coli_moe_read_status(const void* ws, uint32_t* status, void* stream)
@@ -346,6 +402,22 @@ coli_status coli_moe_forward(const coli_moe_dims* dims, const coli_moe_weights* 
         if (!gemm_supported(a)) return COLI_EUNSUPPORTED;
         return cuda_status(gemm_forward(a, s));
     }
+    FusedParams f;
+    if (fused_setup(f, dims, T, 1, ws)) {
+        // decode batch: one launch for the experts and the combine
+        f.route = 0;
+        fused_layer_ptrs(f.layer[0], weights, nullptr);
+        f.x = reinterpret_cast<const float*>(x);
+        f.residual = residual;
+        f.y = y;
+        f.idx = const_cast<int32_t*>(idx);
+        f.w = const_cast<float*>(w);
+        f.union_ids = const_cast<int32_t*>(union_ids);
+        f.n_union = const_cast<int32_t*>(n_union);
+        f.offsets = const_cast<int32_t*>(offsets);
+        f.assign = const_cast<int32_t*>(assign);
+        return cuda_status(fused_launch(f, s));
+    }
     if (!gemv_shape_ok(dims, T)) return COLI_EUNSUPPORTED;
     GemvParams p = gemv_params(dims, weights, reinterpret_cast<const float*>(x), T, w, union_ids,
                                n_union, offsets, assign, residual, y, ws);
@@ -370,6 +442,25 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* we
         return COLI_EINVAL;
     coli_status st = ws_check(dims, T, ws, ws_bytes);
     if (st != COLI_OK) return st;
+    if (dtype == COLI_F32) {
+        FusedParams f;
+        if (fused_setup(f, dims, T, 1, ws)) {
+            // decode batch: the whole layer in one launch
+            f.route = 1;
+            fused_layer_ptrs(f.layer[0], weights, nullptr);
+            f.x = reinterpret_cast<const float*>(x);
+            f.residual = residual;
+            f.y = y;
+            f.idx = idx;
+            f.w = w;
+            f.logits = logits;
+            f.union_ids = union_ids;
+            f.n_union = n_union;
+            f.offsets = offsets;
+            f.assign = assign;
+            return cuda_status(fused_launch(f, (cudaStream_t)stream));
+        }
+    }
     if (dtype == COLI_F32 && !gemv_shape_ok(dims, T)) return COLI_EUNSUPPORTED;
     RouteParams p = route_params(dims, weights->w_router, weights->router_bias, x, dtype, T, idx, w,
                                  logits, ws);
@@ -407,6 +498,48 @@ coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_weights* we
     GemvParams q = gemv_params(dims, weights, nullptr, T, w, union_ids, n_union, offsets, assign,
                                residual, y, ws);
     return run_gemv(1, q, s);
+}
+
+coli_status coli_moe_stack(const coli_moe_dims* dims, const coli_moe_weights* layers,
+                           const float* const* gamma, int32_t n_layers, double eps, const float* x,
+                           int32_t T, int32_t* idx, float* y, void* ws, size_t ws_bytes,
+                           void* stream)
+{
+    if (!dims_ok(dims) || T < 0 || n_layers < 0 || !(eps >= 0.0)) return COLI_EINVAL;
+    if (T == 0 || n_layers == 0) return COLI_OK;
+    if (!layers || !x || !y || !aligned16(x) || !aligned16(y)) return COLI_EINVAL;
+    const size_t xb = (size_t)T * dims->hidden * sizeof(float);
+    if ((const uint8_t*)x < (const uint8_t*)y + xb && (const uint8_t*)y < (const uint8_t*)x + xb)
+        return COLI_EINVAL;   // y may not overlap x
+    for (int32_t l = 0; l < n_layers; l++) {
+        if (!weights_ok(dims, &layers[l], true)) return COLI_EINVAL;
+        if (gamma && gamma[l] && !aligned16(gamma[l])) return COLI_EINVAL;
+    }
+    coli_status st = ws_check(dims, T, ws, ws_bytes);
+    if (st != COLI_OK) return st;
+    const WsLayout W = ws_layout(dims, T);
+    float* chunk_out = reinterpret_cast<float*>((uint8_t*)ws + W.xchunk);
+    cudaStream_t s = (cudaStream_t)stream;
+    const float* in = x;
+    for (int32_t l0 = 0, j = 0; l0 < n_layers; l0 += kFusedMaxLayers, j++) {
+        const int nl = n_layers - l0 < kFusedMaxLayers ? n_layers - l0 : kFusedMaxLayers;
+        FusedParams f;
+        if (!fused_setup(f, dims, T, nl, ws)) return COLI_EUNSUPPORTED;
+        f.norm = 1;
+        f.eps = eps;
+        f.route = 1;
+        for (int l = 0; l < nl; l++)
+            fused_layer_ptrs(f.layer[l], &layers[l0 + l], gamma ? gamma[l0 + l] : nullptr);
+        // re-plan with the normalisation on (the plan does not depend on it)
+        f.x = in;
+        const bool last = l0 + nl >= n_layers;
+        float* out = last ? y : chunk_out + (size_t)(j & 1) * T * dims->hidden;
+        f.y = out;
+        f.idx_layers = idx ? idx + (size_t)l0 * T * dims->top_k : nullptr;
+        if (fused_launch(f, s) != cudaSuccess) return COLI_ECUDA;
+        in = out;
+    }
+    return COLI_OK;
 }
 
 coli_status coli_rmsnorm(int32_t hidden, int32_t T, const float* x, const float* gamma, double eps,

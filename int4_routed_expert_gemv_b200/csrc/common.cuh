@@ -21,7 +21,8 @@ struct WsHeader {
     uint32_t route_ticket;   // router last-block election counter (returns to 0 after use)
     int32_t path;            // last forward path: 0 fp32 GEMV, 1 bf16 grouped GEMM
     uint32_t timeout_site;   // which wait timed out (diagnostics)
-    uint32_t reserved[60];
+    uint32_t launch_gen;     // fused decode launches completed on this workspace
+    uint32_t reserved[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

@@ -1,0 +1,1997 @@
+// Fused decode kernel: whole routed MoE layers in one persistent launch.
+//
+// Per layer and decode batch (T <= 4 tokens) the launch runs the pages' per-token path --
+// the router picks experts, the batch union lists each distinct expert once, the experts
+// run (colibri technical article "colibri 技术解读", section "引擎结构：一个 C 文件，五步
+// token 路径"; README.zh-CN "工作原理 / 绝不为同一次磁盘读取等待两遍", 批量并集) -- and,
+// for a residual stack, keeps the residual stream on the device from layer to layer
+// (README.zh-CN, same section, COLI_CUDA_PIPE=2):
+//
+//   n  = RMSNorm(x)                                   (stacks only)
+//   l  = n . W_r^T + b, top-k, renormalised softmax   (fp64 sums, fp32 logits)
+//   h  = silu(G n) * (U n)     per union expert and the shared expert
+//   y  = residual + D_s h_s + sum_slot w * D_e h_e
+//
+// One CTA per SM, two warp roles:
+//   * a control warp streams every weight the CTA needs -- its share of the router rows,
+//     gate/up row tiles (8 rows of G beside the same 8 rows of U), its rows of each down
+//     matrix -- through a ring of shared-memory slots with the bulk-copy engine, in the order
+//     the consumers use them; router rows and the shared expert do not depend on the
+//     routing, so they stream first.  Between those and the routed experts the same warp
+//     decides the routing (logits from the router partial sums, top-k, union) and
+//     publishes it to the CTA in shared memory.  A block of consecutive rows arrives as
+//     four contiguous chunks whose shared-memory starts are 32 bytes apart modulo 128, and
+//     the four rows a half-warp reads together come from the four chunks, so the reads
+//     hit distinct banks while a copy still moves kilobytes of consecutive rows;
+//   * 12 consumer warps split each row tile's input columns between them and run the int4
+//     dot products on the tensor cores: mma.sync m16n8k32 s8 x s8 -> s32, with the
+//     weights as A (nibble q placed in the high half of a byte, i.e. 16 q, two
+//     instructions per four weights) and the activations as B.  An activation value is
+//     written as X = x * 126 / m = a + b/254 + c/254^2 with balanced int8 digits (m: the
+//     token's largest magnitude for the layer input, the 64-column group's for h); the
+//     three digit planes (and the two tokens of a pair) are the MMA's columns, so one
+//     instruction forms exact integer sums for all of them.  Each group's sums are scaled
+//     by the weight row's fp16 scale in fp32; the planes are combined at the end of the
+//     row.  The last warp to finish a stage sums the warps' partials (SwiGLU into h, or
+//     the routing-weighted combine into the CTA's output rows); nobody waits for it.
+// Work is split statically: router items and gate/up stages over the CTAs, down rows as
+// one contiguous range per CTA, so every CTA combines its output rows over the segments in
+// a fixed order (shared expert, then the union in ascending expert order) and results are
+// reproducible bit for bit.  Cross-CTA dependencies: router partials -> routing (a
+// counter), gate/up -> down (each h value carries the launch and layer it belongs to, so
+// readers check the data itself and writers need no fence), layer output -> next layer
+// (a counter).  Every wait is bounded and marks the status word on time-out, so no launch
+// can hang.
+#include "common.cuh"
+#include "fused.cuh"
+#include "select.cuh"
+
+namespace coli {
+namespace {
+
+constexpr int NCW = 12;               // consumer warps
+constexpr int NCT = NCW * 32;         // consumer threads
+constexpr int NTHR = NCT + 64;        // + the control warp + the reducer warp: 14 warps, at
+                                      // most 4 per SM sub-partition -> 128 registers/thread
+constexpr int kMaxSlots = 8;
+
+// plane weights: A holds 16 q; digits a, b/254, c/254^2
+constexpr float kPf0 = 1.0f / 16.0f;
+constexpr float kPf1 = 1.0f / (16.0f * 254.0f);
+constexpr float kPf2 = 1.0f / (16.0f * 254.0f * 254.0f);
+
+struct Head {
+    uint64_t full[kMaxSlots];
+    uint64_t empty[kMaxSlots];
+    uint64_t route_bar;
+    int dead;
+    uint32_t gen;                // launch generation (h epochs)
+    uint64_t red_full[8];        // partial-sum buffer b: every consumer warp delivered
+    uint64_t red_empty[8];       // partial-sum buffer b: summed, free again
+    double rsq[NCW][kFusedMaxT];
+    double rnorm[kFusedMaxT];
+    float amax[NCW][kFusedMaxT];
+    float xinv[kFusedMaxT];      // 126 / max|x_t| of the layer input (0 for a zero row)
+    float xfac[kFusedMaxT];      // max|x_t| / 126
+    int sh_tok[kFusedMaxT];      // the shared expert's segment: every token, weight 1
+    float sh_wt[kFusedMaxT];
+};
+
+// Routing of one layer as the CTA uses it (shared memory, two copies by layer parity).
+// Segment 0 is the shared expert when there is one, then the union in ascending order.
+struct Table {
+    int* hdr;    // [0] segments, [1] union size
+    int* e;      // expert id (-1: shared)
+    int* cnt;    // tokens of the segment
+    int* base;   // first h row of the segment
+    int* tok;    // [seg][kFusedMaxT] token ids, ascending
+    float* wt;   // [seg][kFusedMaxT] routing weights (1 for the shared expert)
+};
+
+__host__ __device__ constexpr uint32_t table_bytes(int S)
+{
+    return (uint32_t)(2 + 3 * S + 2 * kFusedMaxT * S) * 4u;
+}
+
+__device__ __forceinline__ Table table_at(uint8_t* base, int S)
+{
+    Table t;
+    int* w = reinterpret_cast<int*>(base);
+    t.hdr = w;
+    t.e = w + 2;
+    t.cnt = t.e + S;
+    t.base = t.cnt + S;
+    t.tok = t.base + S;
+    t.wt = reinterpret_cast<float*>(t.tok + kFusedMaxT * S);
+    return t;
+}
+
+// One segment's tokens as a consumer uses them.
+struct Seg {
+    int c, base;
+    const int* tok;     // shared memory
+    const float* wt;
+};
+
+__device__ __forceinline__ Seg seg_of(const Table& tb, int s)
+{
+    Seg g;
+    g.c = tb.cnt[s];
+    g.base = tb.base[s];
+    g.tok = tb.tok + s * kFusedMaxT;
+    g.wt = tb.wt + s * kFusedMaxT;
+    return g;
+}
+
+// ---------------------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ bool timed_out(uint32_t* status)
+{
+    return (*reinterpret_cast<volatile uint32_t*>(status) & DEV_TIMEOUT) != 0u;
+}
+
+__device__ __forceinline__ void give_up(uint32_t* status, uint32_t site, volatile int* dead)
+{
+    if (!timed_out(status)) {
+        set_flag(status, DEV_TIMEOUT);
+        atomicExch(status + 3, site);   // WsHeader::timeout_site
+    }
+    *dead = 1;
+}
+
+// Wait until *p >= target (acquire).  Bounded: after the budget, or once any CTA has timed
+// out, the CTA is marked dead and the wait returns false.
+__device__ __forceinline__ bool gwait(const uint32_t* p, uint32_t target, uint32_t* status, uint32_t site,
+                      volatile int* dead)
+{
+    if (*dead) return false;
+    if (ld_acquire(p) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(128);   // polls leave the issue slots to the working warps
+        if (ld_acquire(p) >= target) return true;
+        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+            give_up(status, site, dead);
+            return false;
+        }
+    }
+}
+
+// mbarrier phase wait that suspends the thread in hardware (up to ~0.1 ms per try) instead
+// of spinning, so waiting warps leave the issue slots to the working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mwait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t site,
+                      volatile int* dead)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*dead) return false;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (*dead) return false;
+        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+            give_up(status, site, dead);
+            return false;
+        }
+    }
+}
+
+// Wait until the shared-memory word *p >= target (another warp of the CTA sets it).
+__device__ __forceinline__ bool swait(const int* p, int target, uint32_t* status, uint32_t site, volatile int* dead)
+{
+    const volatile int* vp = p;
+    if (*vp >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(32);
+        if (*vp >= target) return true;
+        if (*dead) return false;
+        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+            give_up(status, site, dead);
+            return false;
+        }
+    }
+}
+
+// A[16 x 32] (s8, row) x B[32 x 8] (s8, col) + D -> D (s32)
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four packed nibbles pairs -> signed bytes 16 q: even columns (low nibbles) and odd
+// columns (high nibbles) of the word.
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return w & 0xF0F0F0F0u; }
+
+// Round to nearest even for |v| < 2^22: the integer and its float value.
+__device__ __forceinline__ int rint_small(float v, float& vf)
+{
+    const float t = __fadd_rn(v, 12582912.0f);
+    vf = __fsub_rn(t, 12582912.0f);
+    return __float_as_int(t) - 0x4B400000;
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Lane l holds activations 4l..4l+3 of 128 consecutive columns (lanes 0-15 the first
+// 64-column group, 16-31 the second).  Each value becomes three balanced int8 digits of
+// X = x * 126 / m (m = the group's largest magnitude): X ~ a + b/254 + c/254^2, |error| <=
+// 0.5/254^2 + rounding, a in [-126, 126], b, c in [-127, 127].  The lane's three plane
+// words (4 digits each, column order) go to sc[plane * 32 + l]; returns m of its group.
+__device__ __forceinline__ float digits128(float4 v, int lane, uint32_t* sc)
+{
+    float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    const float inv = mx > 0.0f ? 126.0f / mx : 0.0f;
+    const float xs[4] = {v.x, v.y, v.z, v.w};
+    int da[4], db[4], dc[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float X = fminf(fmaxf(xs[i] * inv, -126.0f), 126.0f);
+        float af, bf, cf;
+        da[i] = rint_small(X, af);
+        const float e1 = (X - af) * 254.0f;
+        db[i] = rint_small(e1, bf);
+        const float e2 = (e1 - bf) * 254.0f;
+        dc[i] = rint_small(e2, cf);
+    }
+    sc[lane] = pack4(da[0], da[1], da[2], da[3]);
+    sc[32 + lane] = pack4(db[0], db[1], db[2], db[3]);
+    sc[64 + lane] = pack4(dc[0], dc[1], dc[2], dc[3]);
+    return mx;
+}
+
+// As digits128 with a scale given for the whole row (inv = 126 / max|row|).
+__device__ __forceinline__ void digits128_fixed(float4 v, float inv, int lane, uint32_t* sc)
+{
+    const float xs[4] = {v.x, v.y, v.z, v.w};
+    int da[4], db[4], dc[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float X = fminf(fmaxf(xs[i] * inv, -126.0f), 126.0f);
+        float af, bf, cf;
+        da[i] = rint_small(X, af);
+        const float e1 = (X - af) * 254.0f;
+        db[i] = rint_small(e1, bf);
+        const float e2 = (e1 - bf) * 254.0f;
+        dc[i] = rint_small(e2, cf);
+    }
+    sc[lane] = pack4(da[0], da[1], da[2], da[3]);
+    sc[32 + lane] = pack4(db[0], db[1], db[2], db[3]);
+    sc[64 + lane] = pack4(dc[0], dc[1], dc[2], dc[3]);
+}
+
+// B fragments of 64-column group gl (0/1) of the last digits128 call for the lane
+// (groupID n, threadID tq): plane `plane`, columns 64 gl + 16 tq + 8 j + {0..7} split
+// into even (b[2j]) and odd (b[2j+1]) columns, matching the A side's nibble expansion.
+__device__ __forceinline__ void gather4(const uint32_t* sc, int plane, int gl, int tq,
+                                        uint32_t (&b)[4])
+{
+    const uint4 w = *reinterpret_cast<const uint4*>(sc + plane * 32 + 16 * gl + 4 * tq);
+    b[0] = __byte_perm(w.x, w.y, 0x6420);
+    b[1] = __byte_perm(w.x, w.y, 0x7531);
+    b[2] = __byte_perm(w.z, w.w, 0x6420);
+    b[3] = __byte_perm(w.z, w.w, 0x7531);
+}
+
+// Activation operand of a warp's K range for MMA column tile q (token slots 0 and 1: rows
+// row0 / row1, absent when !p0 / !p1): groups gbase .. gbase+gpw-1 of K columns as B
+// fragments for this lane (groupID n -> slot n >> 2, plane n & 3), every element written.
+// Lane l takes columns 64 (gbase + gi) + 4 l .. +3 of each pair of groups gi, gi + 1; all
+// loads of the call are issued before the first digit is formed.
+//   HEP false: the layer input with one scale per token (inv0 / inv1 = 126 / max|x|),
+//              RMS-normalised first when NORM (n = float(x * r * gamma));
+//   HEP true : SwiGLU activations h stored as (value, epoch) pairs; a pair whose epoch is
+//              not `epoch` is not written yet and is read again (bounded).  Per-group
+//              scales: fac receives m / 126 of the group for the lane's epilogue slot
+//              (threadID >> 1).
+template <int GPWM, int NTM, bool HEP>
+__device__ __forceinline__ void build_tile(const void* row0, const void* row1, bool p0, bool p1,
+                                           float inv0, float inv1, double rn0, double rn1,
+                                           const float* gamma, uint32_t epoch, int gbase, int gpw,
+                                           int q, uint32_t* sc, int lane, uint32_t (&B)[GPWM][NTM][4],
+                                           float (&fac)[GPWM][NTM], uint32_t* status,
+                                           volatile int* dead)
+{
+    constexpr int NP = (GPWM + 1) / 2;
+    const int bslot = lane >> 4, plane = (lane >> 2) & 3, tq = lane & 3, fslot = tq >> 1;
+    const int pl = plane < 3 ? plane : 0;
+    const uint32_t keep = plane < 3 ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+    for (int gi = 0; gi < GPWM; gi++) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) B[gi][q][i] = 0u;
+        fac[gi][q] = 0.0f;
+    }
+#pragma unroll 1
+    for (int sl = 0; sl < 2; sl++) {
+        if (!(sl ? p1 : p0)) continue;   // absent token: zeros
+        const void* row = sl ? row1 : row0;
+        float4 v[NP];
+        bool want[NP];
+#pragma unroll
+        for (int pi = 0; pi < NP; pi++) {
+            const int gi = 2 * pi;
+            want[pi] = gi < gpw && (lane < 16 || gi + 1 < gpw);
+            v[pi] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (HEP) {
+            // (value, epoch) pairs, read until every pair carries this layer's epoch
+            const long long t0 = clock64();
+            bool ok = false;
+            while (!ok) {
+                ok = true;
+#pragma unroll
+                for (int pi = 0; pi < NP; pi++) {
+                    if (want[pi]) {
+                        const uint4* hp = reinterpret_cast<const uint4*>(
+                            reinterpret_cast<const uint2*>(row) + 64 * (gbase + 2 * pi) + 4 * lane);
+                        const uint4 a = __ldcg(hp), b = __ldcg(hp + 1);
+                        ok = ok && a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch;
+                        v[pi] = make_float4(__uint_as_float(a.x), __uint_as_float(a.z),
+                                            __uint_as_float(b.x), __uint_as_float(b.z));
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok && (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles)) {
+                    if (lane == 0) give_up(status, 56, dead);
+                    break;
+                }
+                if (!ok) __nanosleep(256);
+            }
+        } else {
+#pragma unroll
+            for (int pi = 0; pi < NP; pi++)
+                if (want[pi])
+                    v[pi] = __ldcg(reinterpret_cast<const float4*>(
+                        reinterpret_cast<const float*>(row) + 64 * (gbase + 2 * pi) + 4 * lane));
+            {
+                const double r = sl ? rn1 : rn0;
+#pragma unroll
+                for (int pi = 0; pi < NP; pi++) {
+                    const int c0 = 64 * (gbase + 2 * pi) + 4 * lane;
+                    float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+                    if (gamma && want[pi]) gm = __ldg(reinterpret_cast<const float4*>(gamma + c0));
+                    float4& x = v[pi];
+                    x.x = (float)((double)x.x * r * (double)gm.x);
+                    x.y = (float)((double)x.y * r * (double)gm.y);
+                    x.z = (float)((double)x.z * r * (double)gm.z);
+                    x.w = (float)((double)x.w * r * (double)gm.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int pi = 0; pi < NP; pi++) {
+            const int gi = 2 * pi;
+            if (gi < gpw) {
+                float f0 = 0.0f, f1 = 0.0f;
+                if (HEP) {
+                    const float mx = digits128(v[pi], lane, sc);
+                    f0 = __shfl_sync(0xffffffffu, mx, 0) * (1.0f / 126.0f);
+                    f1 = __shfl_sync(0xffffffffu, mx, 16) * (1.0f / 126.0f);
+                } else {
+                    digits128_fixed(v[pi], sl ? inv1 : inv0, lane, sc);
+                }
+                __syncwarp();
+                uint32_t b0[4], b1[4];
+                gather4(sc, pl, 0, tq, b0);
+                gather4(sc, pl, 1, tq, b1);
+                __syncwarp();
+                if (bslot == sl) {
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        B[gi][q][i] = b0[i] & keep;
+                        if (gi + 1 < GPWM) B[gi + 1][q][i] = b1[i] & keep;
+                    }
+                }
+                if (fslot == sl) {
+                    fac[gi][q] = f0;
+                    if (gi + 1 < GPWM) fac[gi + 1][q] = f1;
+                }
+            }
+        }
+    }
+}
+
+// Partial dot products of one row tile (16 MMA rows) over this warp's groups.  ra / rb: the
+// lane's rows g and g + 8 (their group G starts at byte 32 G; the lane's 8 bytes at
+// + 8 threadID), sa / sb: those rows' fp16 scales (one per group).  PERGROUP: multiply each
+// group's sums by fac (per-group activation factors); else the activation factor is
+// applied per token afterwards.
+template <int GPWM, int NTM, bool PERGROUP>
+__device__ __forceinline__ void tile_dot(const uint8_t* ra, const uint8_t* rb, const __half* sa,
+                                         const __half* sb, int gbase, int gpw, uint32_t qmask,
+                                         const uint32_t (&B)[GPWM][NTM][4],
+                                         const float (&fac)[GPWM][NTM], float (&acc)[NTM][4])
+{
+#pragma unroll
+    for (int q = 0; q < NTM; q++)
+#pragma unroll
+        for (int i = 0; i < 4; i++) acc[q][i] = 0.0f;
+    // every warp runs GPWM groups so the groups' loads and MMAs overlap; a warp with fewer
+    // (gpw) re-reads its last group against a zero operand, which adds exactly 0
+#pragma unroll
+    for (int gi = 0; gi < GPWM; gi++) {
+        const int G = gbase + (gi < gpw ? gi : gpw - 1);
+        const uint2 wa = *reinterpret_cast<const uint2*>(ra + 32 * G);
+        const uint2 wb = *reinterpret_cast<const uint2*>(rb + 32 * G);
+        const float s0 = __half2float(sa[G]);
+        const float s1 = __half2float(sb[G]);
+        const uint32_t a00 = nib_lo(wa.x), a01 = nib_lo(wb.x), a02 = nib_hi(wa.x), a03 = nib_hi(wb.x);
+        const uint32_t a10 = nib_lo(wa.y), a11 = nib_lo(wb.y), a12 = nib_hi(wa.y), a13 = nib_hi(wb.y);
+#pragma unroll
+        for (int q = 0; q < NTM; q++) {
+            if ((qmask >> q) & 1u) {
+                int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+                mma_s8(d0, a00, a01, a02, a03, B[gi][q][0], B[gi][q][1]);
+                mma_s8(d1, a10, a11, a12, a13, B[gi][q][2], B[gi][q][3]);
+                const float f0 = PERGROUP ? s0 * fac[gi][q] : s0;
+                const float f1 = PERGROUP ? s1 * fac[gi][q] : s1;
+                acc[q][0] = fmaf((float)(d0[0] + d1[0]), f0, acc[q][0]);
+                acc[q][1] = fmaf((float)(d0[1] + d1[1]), f0, acc[q][1]);
+                acc[q][2] = fmaf((float)(d0[2] + d1[2]), f1, acc[q][2]);
+                acc[q][3] = fmaf((float)(d0[3] + d1[3]), f1, acc[q][3]);
+            }
+        }
+    }
+}
+
+// Combines the planes of the tile's accumulators and writes this warp's partial for
+// (row g, token slot) and (row g + 8, token slot) into red[row][T] (stride T floats).
+// xf: per-slot activation factor (max|x|/126 of the token) or null when the factors were
+// applied per group.
+template <int NTM>
+__device__ __forceinline__ void tile_partials(const float (&acc)[NTM][4], uint32_t qmask, int lane,
+                                              int nslots, float* red, int T, const float* xf)
+{
+    const int g = lane >> 2, t = lane & 3;
+    const float pf0 = (t & 1) ? kPf2 : kPf0, pf1 = (t & 1) ? 0.0f : kPf1;
+#pragma unroll
+    for (int q = 0; q < NTM; q++) {
+        if ((qmask >> q) & 1u) {
+            float f = 1.0f;
+            if (xf) {
+                const int sl = 2 * q + (t >> 1);
+                f = sl < T ? xf[sl] : 0.0f;
+            }
+            float v0 = (acc[q][0] * pf0 + acc[q][1] * pf1) * f;
+            float v1 = (acc[q][2] * pf0 + acc[q][3] * pf1) * f;
+            v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+            v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+            const int s = 2 * q + (t >> 1);
+            if ((t & 1) == 0 && s < nslots) {
+                red[g * T + s] = v0;
+                red[(g + 8) * T + s] = v1;
+            }
+        }
+    }
+}
+
+// ---- one-token gate/up in group pairs ------------------------------------------------
+// A lane loads 16 bytes of a row (32 columns: lanes t < 2 of group 2P, t >= 2 of group
+// 2P + 1) and feeds four MMAs.  The activation operand is block diagonal: columns 0-3 of
+// the MMA are the digit planes of group 2P and only the k-slots of lanes t < 2 carry them,
+// columns 4-7 those of group 2P + 1 from lanes t >= 2, so one accumulator holds both
+// groups' sums and a lane's two columns belong to a single group (one scale per row).
+
+// Operand of pair P of the warp's groups for the layer input (token 0): Bp[pair][8] in the
+// register array B[2P + (r >> 2)][0][r & 3], r = 0..7 (MMA j uses registers 2j, 2j + 1).
+template <int GPWM, int NTM>
+__device__ __forceinline__ void build_x_pairs(const float* row, float inv, double rn,
+                                              const float* gamma, int gbase, int gpw, uint32_t* sc,
+                                              int lane, uint32_t (&B)[GPWM][NTM][4])
+{
+    constexpr int NP = GPWM / 2;
+    const int n = lane >> 2, tq = lane & 3, plane = n & 3;
+    const int pl = plane < 3 ? plane : 0;
+    const bool mine = plane < 3 && (n >> 2) == (tq >> 1);
+    float4 v[NP];
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++)
+        v[pi] = 2 * pi < gpw ? __ldcg(reinterpret_cast<const float4*>(row + 64 * (gbase + 2 * pi) + 4 * lane))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    // n = float(x * r * gamma); r = 1 and gamma = 1 leave a plain input exactly as it is
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++) {
+        const int c0 = 64 * (gbase + 2 * pi) + 4 * lane;
+        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (gamma && 2 * pi < gpw) gm = __ldg(reinterpret_cast<const float4*>(gamma + c0));
+        float4& x = v[pi];
+        x.x = (float)((double)x.x * rn * (double)gm.x);
+        x.y = (float)((double)x.y * rn * (double)gm.y);
+        x.z = (float)((double)x.z * rn * (double)gm.z);
+        x.w = (float)((double)x.w * rn * (double)gm.w);
+    }
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++) {
+        digits128_fixed(v[pi], inv, lane, sc);
+        __syncwarp();
+        // words 8 tq .. 8 tq + 7 of the plane: columns 32 tq .. 32 tq + 31 of the pair
+        const uint4 w0 = *reinterpret_cast<const uint4*>(sc + pl * 32 + 8 * tq);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(sc + pl * 32 + 8 * tq + 4);
+        __syncwarp();
+        const uint32_t keep = mine ? 0xFFFFFFFFu : 0u;
+        uint32_t r[8];
+        r[0] = __byte_perm(w0.x, w0.y, 0x6420);
+        r[1] = __byte_perm(w0.x, w0.y, 0x7531);
+        r[2] = __byte_perm(w0.z, w0.w, 0x6420);
+        r[3] = __byte_perm(w0.z, w0.w, 0x7531);
+        r[4] = __byte_perm(w1.x, w1.y, 0x6420);
+        r[5] = __byte_perm(w1.x, w1.y, 0x7531);
+        r[6] = __byte_perm(w1.z, w1.w, 0x6420);
+        r[7] = __byte_perm(w1.z, w1.w, 0x7531);
+#pragma unroll
+        for (int i = 0; i < 8; i++) B[2 * pi + (i >> 2)][0][i & 3] = r[i] & keep;
+    }
+}
+
+// Operand of the warp's group pairs of h rows (one token; (value, epoch) pairs read until
+// they carry `epoch`, bounded), per-group scales: the lane's factor m / 126 of its group
+// (2 P + (threadID >> 1)) in fac[2 P][0].
+template <int GPWM, int NTM>
+__device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, int gbase, uint32_t* sc,
+                                              int lane, uint32_t (&B)[GPWM][NTM][4],
+                                              float (&fac)[GPWM][NTM], uint32_t* status,
+                                              volatile int* dead)
+{
+    constexpr int NP = GPWM / 2;
+    const int n = lane >> 2, tq = lane & 3, plane = n & 3;
+    const int pl = plane < 3 ? plane : 0;
+    const bool mine = plane < 3 && (n >> 2) == (tq >> 1);
+    float4 v[NP];
+    const long long t0 = clock64();
+    bool ok = false;
+    while (!ok) {
+        ok = true;
+#pragma unroll
+        for (int pi = 0; pi < NP; pi++) {
+            const uint4* hp = reinterpret_cast<const uint4*>(row + 64 * (gbase + 2 * pi) + 4 * lane);
+            const uint4 a = __ldcg(hp), b = __ldcg(hp + 1);
+            ok = ok && a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch;
+            v[pi] = make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x),
+                                __uint_as_float(b.z));
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles)) {
+            if (lane == 0) give_up(status, 56, dead);
+            break;
+        }
+        if (!ok) __nanosleep(256);
+    }
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++) {
+        const float mx = digits128(v[pi], lane, sc);
+        const float m0 = __shfl_sync(0xffffffffu, mx, 0), m1 = __shfl_sync(0xffffffffu, mx, 16);
+        __syncwarp();
+        const uint4 w0 = *reinterpret_cast<const uint4*>(sc + pl * 32 + 8 * tq);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(sc + pl * 32 + 8 * tq + 4);
+        __syncwarp();
+        const uint32_t keep = mine ? 0xFFFFFFFFu : 0u;
+        uint32_t r[8];
+        r[0] = __byte_perm(w0.x, w0.y, 0x6420);
+        r[1] = __byte_perm(w0.x, w0.y, 0x7531);
+        r[2] = __byte_perm(w0.z, w0.w, 0x6420);
+        r[3] = __byte_perm(w0.z, w0.w, 0x7531);
+        r[4] = __byte_perm(w1.x, w1.y, 0x6420);
+        r[5] = __byte_perm(w1.x, w1.y, 0x7531);
+        r[6] = __byte_perm(w1.z, w1.w, 0x6420);
+        r[7] = __byte_perm(w1.z, w1.w, 0x7531);
+#pragma unroll
+        for (int i = 0; i < 8; i++) B[2 * pi + (i >> 2)][0][i & 3] = r[i] & keep;
+        fac[2 * pi][0] = ((tq >> 1) ? m1 : m0) * (1.0f / 126.0f);
+        fac[2 * pi + 1][0] = 0.0f;
+    }
+}
+
+// Digits of one token's h row (I columns), once per CTA: warp w digitizes group pairs w,
+// w + NCW, ... into the compact buffer dig (plane p: I bytes at p * I, column order) and the
+// group factors m / 126 into fac.  (value, epoch) pairs are read until they carry `epoch`.
+__device__ __forceinline__ void digitize_h_row(const uint2* row, uint32_t epoch, int I, int warp, int lane,
+                                               uint32_t* sc, uint32_t* dig, float* fac,
+                                               uint32_t* status, volatile int* dead)
+{
+    const int npairs = I / 128;
+    for (int pp = warp; pp < npairs; pp += NCW) {
+        const uint4* hp = reinterpret_cast<const uint4*>(row + 128 * pp + 4 * lane);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        const long long t0 = clock64();
+        while (true) {
+            const uint4 a = __ldcg(hp), b = __ldcg(hp + 1);
+            const bool ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
+            v = make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x), __uint_as_float(b.z));
+            if (ok) break;
+            if (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+                if (lane == 0) give_up(status, 56, dead);
+                break;
+            }
+            __nanosleep(256);
+        }
+        const float mx = digits128(v, lane, sc);
+        __syncwarp();
+#pragma unroll
+        for (int pl = 0; pl < 3; pl++) dig[pl * (I / 4) + 32 * pp + lane] = sc[pl * 32 + lane];
+        if (lane == 0) fac[2 * pp] = mx * (1.0f / 126.0f);
+        if (lane == 16) fac[2 * pp + 1] = mx * (1.0f / 126.0f);
+        __syncwarp();
+    }
+}
+
+// Pair-form operand of the warp's groups from the compact digits of digitize_h_row.
+template <int GPWM, int NTM>
+__device__ __forceinline__ void gather_h_pairs(const uint32_t* dig, const float* facs, int I, int gbase,
+                                               int lane, uint32_t (&B)[GPWM][NTM][4],
+                                               float (&fac)[GPWM][NTM])
+{
+    constexpr int NP = GPWM / 2;
+    const int n = lane >> 2, tq = lane & 3, plane = n & 3;
+    const int pl = plane < 3 ? plane : 0;
+    const uint32_t keep = (plane < 3 && (n >> 2) == (tq >> 1)) ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++) {
+        const uint32_t* src = dig + pl * (I / 4) + 32 * (gbase / 2 + pi) + 8 * tq;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(src);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(src + 4);
+        uint32_t r[8];
+        r[0] = __byte_perm(w0.x, w0.y, 0x6420);
+        r[1] = __byte_perm(w0.x, w0.y, 0x7531);
+        r[2] = __byte_perm(w0.z, w0.w, 0x6420);
+        r[3] = __byte_perm(w0.z, w0.w, 0x7531);
+        r[4] = __byte_perm(w1.x, w1.y, 0x6420);
+        r[5] = __byte_perm(w1.x, w1.y, 0x7531);
+        r[6] = __byte_perm(w1.z, w1.w, 0x6420);
+        r[7] = __byte_perm(w1.z, w1.w, 0x7531);
+#pragma unroll
+        for (int i = 0; i < 8; i++) B[2 * pi + (i >> 2)][0][i & 3] = r[i] & keep;
+        fac[2 * pi][0] = facs[gbase + 2 * pi + (tq >> 1)];
+        fac[2 * pi + 1][0] = 0.0f;
+    }
+}
+
+// Partial sums of one row tile over the warp's group pairs: ra / rb the lane's rows g and
+// g + 8 (pair P at byte 64 P, the lane's 16 bytes at + 16 threadID), sa / sb their scales.
+// PG: per-group activation factors (h), the lane's in fac[2 P][0] for pair P.
+template <int GPWM, int NTM, bool PG>
+__device__ __forceinline__ void tile_dot_pairs(const uint8_t* ra, const uint8_t* rb, const __half* sa,
+                                               const __half* sb, int gbase, int lane,
+                                               const uint32_t (&B)[GPWM][NTM][4],
+                                               const float (&fac)[GPWM][NTM], float (&acc)[4])
+{
+    constexpr int NP = GPWM / 2;
+    static_assert(GPWM == 4 || GPWM == 8, "pair tiles: 4 or 8 groups per warp");
+    const int half = (lane & 3) >> 1;
+    // the rows' scales of the warp's groups in one read each (16 or 8 bytes, aligned: the
+    // warp's first group is a multiple of GPWM)
+    uint32_t swa[NP], swb[NP];
+    if (GPWM == 8) {
+        const uint4 a = *reinterpret_cast<const uint4*>(sa + gbase);
+        const uint4 b = *reinterpret_cast<const uint4*>(sb + gbase);
+        swa[0] = a.x; swa[1 % NP] = a.y; swa[2 % NP] = a.z; swa[3 % NP] = a.w;
+        swb[0] = b.x; swb[1 % NP] = b.y; swb[2 % NP] = b.z; swb[3 % NP] = b.w;
+    } else {
+        const uint2 a = *reinterpret_cast<const uint2*>(sa + gbase);
+        const uint2 b = *reinterpret_cast<const uint2*>(sb + gbase);
+        swa[0] = a.x; swa[1 % NP] = a.y;
+        swb[0] = b.x; swb[1 % NP] = b.y;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) acc[i] = 0.0f;
+#pragma unroll
+    for (int pi = 0; pi < NP; pi++) {
+        const int G = gbase + 2 * pi;
+        const uint4 wa = *reinterpret_cast<const uint4*>(ra + 32 * G);
+        const uint4 wb = *reinterpret_cast<const uint4*>(rb + 32 * G);
+        float s0 = __half2float(__ushort_as_half((unsigned short)(half ? swa[pi] >> 16 : swa[pi] & 0xFFFFu)));
+        float s1 = __half2float(__ushort_as_half((unsigned short)(half ? swb[pi] >> 16 : swb[pi] & 0xFFFFu)));
+        if (PG) {
+            s0 *= fac[2 * pi][0];
+            s1 *= fac[2 * pi][0];
+        }
+        const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
+        int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint32_t b0 = B[2 * pi + (j >> 1)][0][2 * (j & 1)];
+            const uint32_t b1 = B[2 * pi + (j >> 1)][0][2 * (j & 1) + 1];
+            if (j < 2) mma_s8(d0, nib_lo(xa[j]), nib_lo(xb[j]), nib_hi(xa[j]), nib_hi(xb[j]), b0, b1);
+            else mma_s8(d1, nib_lo(xa[j]), nib_lo(xb[j]), nib_hi(xa[j]), nib_hi(xb[j]), b0, b1);
+        }
+        acc[0] = fmaf((float)(d0[0] + d1[0]), s0, acc[0]);
+        acc[1] = fmaf((float)(d0[1] + d1[1]), s0, acc[1]);
+        acc[2] = fmaf((float)(d0[2] + d1[2]), s1, acc[2]);
+        acc[3] = fmaf((float)(d0[3] + d1[3]), s1, acc[3]);
+    }
+}
+
+// Row sums of a pair-mode tile: every lane of a row holds two planes of one group; the
+// four lanes together hold the whole row (both groups, all planes).  Writes red[g] and
+// red[g + 8] (one token), scaled by the token's activation factor.
+__device__ __forceinline__ void tile_partials_pairs(const float (&acc)[4], int lane, float* red, float xf)
+{
+    const int g = lane >> 2, t = lane & 3;
+    const float pf0 = (t & 1) ? kPf2 : kPf0, pf1 = (t & 1) ? 0.0f : kPf1;
+    float v0 = acc[0] * pf0 + acc[1] * pf1;
+    float v1 = acc[2] * pf0 + acc[3] * pf1;
+    v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+    v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+    v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+    v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+    if (t == 0) {
+        red[g] = v0 * xf;
+        red[g + 8] = v1 * xf;
+    }
+}
+
+// Partial sums go through a ring of kRedBufs buffers: stage cs (every gate/up and down
+// stage, in the consumers' order) writes buffer cs % kRedBufs; each consumer warp arrives on
+// the buffer's full barrier after writing its part; the reducer warp waits for it, sums
+// (SwiGLU into h, or the routing-weighted combine into the CTA's output rows, in stage
+// order) and arrives on the buffer's empty barrier, which a consumer waits for before it
+// writes the buffer again.  No compute warp ever waits for another one.
+constexpr int kRedBufs = 6;
+
+__device__ __forceinline__ void red_wait_free(Head& hd, uint32_t cs, uint32_t* status,
+                                              volatile int* dead, int lane)
+{
+    if (cs >= (uint32_t)kRedBufs)
+        mwait(&hd.red_empty[cs % kRedBufs], ((cs / kRedBufs) - 1u) & 1u, status, 57, dead);
+}
+
+__device__ __forceinline__ void red_deliver(Head& hd, uint32_t cs, int lane)
+{
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&hd.red_full[cs % kRedBufs]);
+}
+
+// blob section offsets (bytes)
+struct BlobOff {
+    uint64_t gq, uq, dq, gs, us, ds;
+};
+__device__ __forceinline__ BlobOff blob_off(int H, int I)
+{
+    const uint64_t IH = (uint64_t)I * H;
+    BlobOff o;
+    o.gq = 0;
+    o.uq = IH / 2;
+    o.dq = IH;
+    o.gs = 3 * IH / 2;
+    o.us = o.gs + IH / 32;
+    o.ds = o.us + IH / 32;
+    return o;
+}
+
+// Top-k of lt[0..E) in shared memory, as select.cuh's topk_warp_keys (keys, ties to the
+// lower index): lane s < k returns selection s.
+template <int MAXPL>
+__device__ __forceinline__ void topk_smem(const float* lt, int E, int k, int lane, int& e_out,
+                                          uint32_t& key_out)
+{
+    uint32_t key[MAXPL];
+#pragma unroll
+    for (int i = 0; i < MAXPL; i++) {
+        const int e = lane + 32 * i;
+        key[i] = (e < E) ? order_key(lt[e]) : 0u;
+    }
+    uint32_t mine = 0u;
+    int mine_e = 0;
+    for (int s = 0; s < k; s++) {
+        uint32_t bk = key[0];
+        int bi = 0;
+#pragma unroll
+        for (int i = 1; i < MAXPL; i++)
+            if (key[i] > bk) {
+                bk = key[i];
+                bi = i;
+            }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == m) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+        const uint32_t e = __reduce_min_sync(0xffffffffu, cand);
+        if ((int)(e & 31u) == lane) {
+#pragma unroll
+            for (int i = 0; i < MAXPL; i++)
+                if (i == (int)(e >> 5)) key[i] = 0u;
+        }
+        if (lane == s) {
+            mine = m;
+            mine_e = (int)e;
+        }
+    }
+    e_out = mine_e;
+    key_out = mine;
+}
+
+// Exclusive prefix sum over the warp's lanes.
+__device__ __forceinline__ int warp_excl_scan(int v, int lane)
+{
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    return x - v;
+}
+
+// Union of sel[t * k + s] (T * k <= 128 assignments, each token's experts distinct and in
+// [0, E)): writes the routed segments of the table (after n_shared leading segments) and,
+// when `out` is set, union_ids / n_union / offsets / assign.  bits: T * 32 words scratch.
+__device__ __forceinline__ void build_union(const int* sel, const float* selw, int T, int k, int E, int ns,
+                            uint32_t* bits, Table tb, bool out, const FusedParams& p, int lane)
+{
+    const int nw = (E + 31) / 32;
+    const int n = T * k;
+    for (int i = lane; i < kFusedMaxT * 32; i += 32) bits[i] = 0u;
+    __syncwarp();
+    for (int a = lane; a < n; a += 32) {
+        const int e = sel[a];
+        atomicOr(&bits[(a / k) * 32 + (e >> 5)], 1u << (e & 31));
+    }
+    __syncwarp();
+    // per word w (lane w < nw): union word, and per token the prefix popcounts
+    uint32_t uw = 0u;
+    int pre_t[kFusedMaxT];
+    int cnt_below = 0;   // assignments with a smaller expert word, all tokens
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; t++) {
+        const uint32_t bw = (t < T && lane < nw) ? bits[t * 32 + lane] : 0u;
+        uw |= bw;
+        pre_t[t] = warp_excl_scan(__popc(bw), lane);
+        cnt_below += pre_t[t];
+    }
+    const int upre = warp_excl_scan(__popc(uw), lane);
+    const int nu = __shfl_sync(0xffffffffu, upre + __popc(uw), 31);
+    for (int a0 = 0; a0 < n; a0 += 32) {
+        const int a = a0 + lane;
+        const bool valid = a < n;
+        const int e = valid ? sel[a] : 0;
+        const int t = valid ? a / k : 0;
+        const int w = e >> 5;
+        const uint32_t below = (1u << (e & 31)) - 1u;
+        const int up_w = __shfl_sync(0xffffffffu, upre, w);
+        const uint32_t uw_w = __shfl_sync(0xffffffffu, uw, w);
+        int off = __shfl_sync(0xffffffffu, cnt_below, w);
+        int before_t = 0, count = 0;
+#pragma unroll
+        for (int tt = 0; tt < kFusedMaxT; tt++) {
+            if (tt < T) {
+                const uint32_t bw = bits[tt * 32 + w];
+                off += __popc(bw & below);
+                const int hit = (bw >> (e & 31)) & 1;
+                count += hit;
+                if (tt < t) before_t += hit;
+            }
+        }
+        if (valid) {
+            const int u = up_w + __popc(uw_w & below);
+            const int rank = off + before_t;
+            const int seg = ns + u;
+            if (before_t == 0) {
+                tb.e[seg] = e;
+                tb.cnt[seg] = count;
+                tb.base[seg] = off;
+                if (out) {
+                    p.union_ids[u] = e;
+                    p.offsets[u] = off;
+                }
+            }
+            tb.tok[seg * kFusedMaxT + before_t] = t;
+            tb.wt[seg * kFusedMaxT + before_t] = selw[a];
+            if (out) p.assign[rank] = a;
+        }
+    }
+    if (out) {
+        for (int q = nu + lane; q <= E; q += 32) {
+            if (q < E) p.union_ids[q] = -1;
+            p.offsets[q] = n;
+        }
+        if (lane == 0) *p.n_union = nu;
+    }
+    if (lane == 0) {
+        tb.hdr[0] = ns + nu;
+        tb.hdr[1] = nu;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------------------
+
+// Per-CTA constants shared by the roles.
+struct Ctx {
+    Head* hd;
+    volatile int* dead;
+    uint8_t* ring;
+    float* red;
+    float* yacc;
+    uint8_t* rt_base;
+    uint32_t tbytes;
+    int S;
+    int tid, warp, lane, b, G;
+    int r0, r1, nrows, ntd;
+    int ri0, ri1;          // router items of the CTA (contiguous)
+    int n_ritems;
+    BlobOff bo;
+};
+
+// down rows of the CTA in four chunks: chunk q = rows [dcs(q), dcs(q + 1)) of its range
+__device__ __forceinline__ int dcs(const Ctx& c, int q) { return (q * c.nrows) >> 2; }
+
+__device__ __forceinline__ Table layer_table(const Ctx& c, int l)
+{
+    return table_at(c.rt_base + (l & 1) * c.tbytes, c.S);
+}
+
+__device__ __forceinline__ uint32_t* layer_cnt(const FusedParams& p, int l)
+{
+    return p.cnt + 1 + l * kCntPerLayer;
+}
+
+__device__ __forceinline__ uint32_t h_epoch(const Ctx& c, int l)
+{
+    return c.hd->gen * 32u + (uint32_t)l + 1u;
+}
+
+// ----------------------------- control warp: the weight stream --------------------------
+struct Stream {
+    uint32_t it;
+    uint64_t pol;
+};
+
+__device__ __forceinline__ uint8_t* slot_begin(const FusedParams& p, const Ctx& c, Stream& st,
+                                               uint32_t bytes, uint64_t*& bar)
+{
+    const uint32_t s = st.it % (uint32_t)p.nslot;
+    mwait(&c.hd->empty[s], ((st.it / (uint32_t)p.nslot) & 1u) ^ 1u, p.status, 31, c.dead);
+    bar = &c.hd->full[s];
+    mbar_arrive_expect_tx(bar, bytes);
+    st.it++;
+    return c.ring + (size_t)s * p.slot_bytes;
+}
+
+// this CTA's router items: items [ri0, ri1) of the E x RC item list, item i = columns
+// (i % RC) * RKc .. of row i / RC, i.e. floats i * RKc .. of the row-major router matrix
+__device__ __forceinline__ void issue_router(const FusedParams& p, const Ctx& c, Stream& st, const FusedLayer& ly)
+{
+    const uint32_t bytes = (uint32_t)(c.ri1 - c.ri0) * (uint32_t)p.RKc * 4u;
+    uint64_t* bar;
+    uint8_t* dst = slot_begin(p, c, st, bytes, bar);
+    bulk_g2s(dst, ly.w_router + (size_t)c.ri0 * p.RKc, bytes, bar);
+}
+
+// gate/up stage of `ntl` row tiles (8 intermediate rows each) from row i0: the 8 ntl rows of
+// G as four chunks of 2 ntl rows (chunk q at q * gu_chunk), the same rows of U after them,
+// then the G scales and the U scales of the rows
+__device__ __forceinline__ void issue_gu(const FusedParams& p, const Ctx& c, Stream& st, const uint8_t* blob, int stage)
+{
+    const int H = p.H, i0 = stage * 8 * p.NTSg;
+    const int ntl = min(p.NTSg, (p.I - i0) / 8);
+    const uint32_t rowb = (uint32_t)H / 2, cr = 2u * ntl;
+    const uint32_t scb = 8u * ntl * ((uint32_t)H / 32u);
+    uint64_t* bar;
+    uint8_t* dst = slot_begin(p, c, st, 8u * cr * rowb + 2u * scb, bar);
+    for (int q = 0; q < 4; q++) {
+        const uint64_t r = (uint64_t)i0 + q * cr;
+        bulk_g2s_hint(dst + (size_t)q * p.gu_chunk, blob + c.bo.gq + r * rowb, cr * rowb, bar, st.pol);
+        bulk_g2s_hint(dst + (size_t)(4 + q) * p.gu_chunk, blob + c.bo.uq + r * rowb, cr * rowb, bar, st.pol);
+    }
+    bulk_g2s_hint(dst + p.gu_gsc, blob + c.bo.gs + (uint64_t)i0 * (H / 32), scb, bar, st.pol);
+    bulk_g2s_hint(dst + p.gu_usc, blob + c.bo.us + (uint64_t)i0 * (H / 32), scb, bar, st.pol);
+}
+
+// down stage: the CTA's rows r0..r1 of D in four chunks (chunk q at q * d_chunk), then
+// their scales from the 16-byte boundary at or below row r0's first scale
+__device__ __forceinline__ void issue_down(const FusedParams& p, const Ctx& c, Stream& st, const uint8_t* blob)
+{
+    const int I = p.I;
+    const uint32_t rowb = (uint32_t)I / 2;
+    const uint64_t s0 = (uint64_t)c.r0 * (I / 32), s1 = (uint64_t)c.r1 * (I / 32);
+    const uint64_t a0 = s0 & ~15ull, a1 = (s1 + 15) & ~15ull;
+    uint64_t* bar;
+    uint8_t* dst = slot_begin(p, c, st, (uint32_t)c.nrows * rowb + (uint32_t)(a1 - a0), bar);
+    for (int q = 0; q < 4; q++) {
+        const int n = dcs(c, q + 1) - dcs(c, q);
+        if (n > 0)
+            bulk_g2s_hint(dst + (size_t)q * p.d_chunk,
+                          blob + c.bo.dq + (uint64_t)(c.r0 + dcs(c, q)) * rowb, (uint32_t)n * rowb,
+                          bar, st.pol);
+    }
+    bulk_g2s_hint(dst + p.d_sc_off, blob + c.bo.ds + a0, (uint32_t)(a1 - a0), bar, st.pol);
+}
+
+// ----------------------------- control warp: routing ------------------------------------
+// Renormalised softmax weight of selection `lane` (< k) from the order keys held by lanes
+// 0..k-1 (descending): exp(l - l_max) / sum, in fp32 (exp to a few ulp, far inside the
+// 1e-6 bar on the weights).
+__device__ __forceinline__ float topk_weight_f(uint32_t key, int k, int lane)
+{
+    const float lmax = key_float(__shfl_sync(0xffffffffu, key, 0));
+    const float ex = lane < k ? expf(key_float(key) - lmax) : 0.0f;
+    float z = ex;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    return ex / z;
+}
+
+// Routing of layer l: logits from the router partial sums (summed in chunk order) into
+// lt [T][E], top-k and weights per token, then the union into table tb.  `dry`: the same
+// code on whatever the buffers hold (run early, while the control warp would wait anyway,
+// so the real pass finds its instructions cached); it writes nothing but tb and scratch.
+__device__ __forceinline__ void route_compute(const FusedParams& p, const Ctx& c, int l, Table tb, bool dry)
+{
+    const int T = p.T, E = p.E, k = p.k, ns = p.n_shared, lane = c.lane;
+    const FusedLayer& ly = p.layer[l];
+    float* lt = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_scratch +
+                                         NCW * 96 * 4);
+    int* sel = reinterpret_cast<int*>(lt + T * E);
+    float* selw = reinterpret_cast<float*>(sel + T * k);
+    uint32_t* bits = reinterpret_cast<uint32_t*>(selw + T * k);
+    const bool out = c.b == 0 && !dry;
+    for (int t = 0; t < T; t++) {
+        for (int e0 = 0; e0 < E; e0 += 32 * 2) {
+            double part[2][8];
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const int e = e0 + 32 * i + lane;
+#pragma unroll
+                for (int cc = 0; cc < 8; cc++)
+                    part[i][cc] = (e < E && cc < p.RC) ? __ldcg(p.rpart + ((size_t)t * E + e) * p.RC + cc) : 0.0;
+            }
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const int e = e0 + 32 * i + lane;
+                if (e < E) {
+                    double sum = 0.0;
+#pragma unroll
+                    for (int cc = 0; cc < 8; cc++)
+                        if (cc < p.RC) sum += part[i][cc];
+                    if (ly.bias) sum += (double)__ldg(ly.bias + e);
+                    const float v = (float)sum;
+                    if (!dry && !isfinite(v)) set_flag(p.status, DEV_NONFINITE);
+                    lt[t * E + e] = v;
+                    if (out && p.logits) p.logits[(size_t)t * E + e] = v;
+                }
+            }
+        }
+    }
+    __syncwarp();
+    for (int t = 0; t < T; t++) {
+        int e_sel;
+        uint32_t key;
+        if (E <= 256) topk_smem<8>(lt + t * E, E, k, lane, e_sel, key);
+        else topk_smem<32>(lt + t * E, E, k, lane, e_sel, key);
+        const float wv = topk_weight_f(key, k, lane);
+        if (lane < k) {
+            sel[t * k + lane] = e_sel;
+            selw[t * k + lane] = wv;
+            if (out && p.idx) p.idx[(size_t)t * k + lane] = e_sel;
+            if (out && p.w) p.w[(size_t)t * k + lane] = wv;
+            if (out && p.idx_layers) p.idx_layers[((size_t)l * T + t) * k + lane] = e_sel;
+        }
+    }
+    __syncwarp();
+    build_union(sel, selw, T, k, E, ns, bits, tb, out && p.union_ids != nullptr, p, lane);
+    __syncwarp();
+}
+
+__device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, int l)
+{
+    const int T = p.T, E = p.E, k = p.k, ns = p.n_shared, lane = c.lane;
+    const Table tb = layer_table(c, l);
+    uint32_t* lc = layer_cnt(p, l);
+    if (p.route) {
+        if (lane == 0) gwait(&lc[0], (uint32_t)c.n_ritems, p.status, 41, c.dead);
+        __syncwarp();
+        route_compute(p, c, l, tb, false);
+    } else {
+        // given routing (forward call): union_ids / n_union / offsets / assign / w
+        int nu = __ldcg(p.n_union);
+        if (nu < 0 || nu > min(E, T * k)) {
+            if (lane == 0) set_flag(p.status, DEV_BAD_INDEX);
+            nu = max(0, min(nu, min(E, T * k)));
+        }
+        for (int u = lane; u < nu; u += 32) {
+            const int seg = ns + u;
+            int e = __ldcg(p.union_ids + u);
+            int o0 = __ldcg(p.offsets + u), o1 = __ldcg(p.offsets + u + 1);
+            const bool bad = e < 0 || e >= E || o0 < 0 || o1 > T * k || o1 - o0 < 1 || o1 - o0 > T;
+            if (bad) {
+                set_flag(p.status, DEV_BAD_INDEX);
+                e = min(max(e, 0), E - 1);
+                o1 = o0 = 0;
+            }
+            tb.e[seg] = e;
+            tb.cnt[seg] = o1 - o0;
+            tb.base[seg] = o0;
+            for (int m = 0; m < o1 - o0; m++) {
+                int a = __ldcg(p.assign + o0 + m);
+                if (a < 0 || a >= T * k) {
+                    set_flag(p.status, DEV_BAD_INDEX);
+                    a = 0;
+                }
+                tb.tok[seg * kFusedMaxT + m] = a / k;
+                tb.wt[seg * kFusedMaxT + m] = __ldcg(p.w + a);
+            }
+        }
+        if (lane == 0) {
+            tb.hdr[0] = ns + nu;
+            tb.hdr[1] = nu;
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.hd->route_bar);
+}
+
+// The control warp's order of stages (the consumers follow the same order): router items,
+// the shared expert's gate/up stages of this CTA and its down rows, [routing], the routed
+// gate/up stages of this CTA (one round-robin sequence over all segments' stages), the
+// routed down rows in union order.
+__device__ __forceinline__ void control_warp(const FusedParams& p, const Ctx& c)
+{
+    Stream st;
+    st.it = 0;
+    st.pol = policy_evict_first();
+    const int ns = p.n_shared;
+    for (int l = 0; l < p.L; l++) {
+        const FusedLayer& ly = p.layer[l];
+        if (c.lane == 0) {
+            if (c.ri1 > c.ri0) issue_router(p, c, st, ly);
+            if (ns) {
+                for (int gi = c.b; gi < p.SPS; gi += c.G) issue_gu(p, c, st, ly.shared, gi);
+                if (c.nrows > 0) issue_down(p, c, st, ly.shared);
+            }
+        }
+        __syncwarp();
+        if (l == 0) {
+            pdl_wait();
+            // warm the routing code path while the router items are still being computed
+            if (p.route && p.L > 0) route_compute(p, c, l, layer_table(c, l + 1), true);
+        }
+        route_layer(p, c, l);
+        if (c.lane == 0) {
+            const Table tb = layer_table(c, l);
+            const int nseg = tb.hdr[0];
+            int gi = c.b;
+            while (gi < ns * p.SPS) gi += c.G;
+            for (; gi < nseg * p.SPS; gi += c.G) {
+                const int s = gi / p.SPS;
+                issue_gu(p, c, st, ly.experts + (uint64_t)tb.e[s] * ly.stride, gi - s * p.SPS);
+            }
+            if (c.nrows > 0)
+                for (int s = ns; s < nseg; s++) issue_down(p, c, st, ly.experts + (uint64_t)tb.e[s] * ly.stride);
+        }
+        __syncwarp();
+    }
+    // drain: every issued copy has landed before the CTA may exit (bounded)
+    if (c.lane == 0) {
+        const uint32_t n_last = st.it < (uint32_t)p.nslot ? st.it : (uint32_t)p.nslot;
+        for (uint32_t q = 0; q < n_last; q++) {
+            const uint32_t last = st.it - 1 - q;
+            const uint32_t s = last % (uint32_t)p.nslot;
+            const uint32_t par = (last / (uint32_t)p.nslot) & 1u;
+            if (!mbar_try_wait(&c.hd->full[s], par)) {
+                const long long t0 = clock64();
+                while (!mbar_try_wait(&c.hd->full[s], par) && clock64() - t0 < kWaitBudgetCycles) {
+                }
+            }
+        }
+    }
+}
+
+// ----------------------------- consumers ------------------------------------------------
+struct Cons {
+    uint32_t it;    // ring position (the control warp's order)
+    uint32_t cs;    // reduction stages
+    uint32_t ds;    // down stages (h digit buffer parity)
+    uint32_t* sc;   // this warp's digit scratch (96 words)
+    int g_rs, g_kw, gbase_g, gpw_g;   // gate/up: row slot, K slot, its groups
+    int d_rs, d_kw, gbase_d, gpw_d;   // down
+};
+
+__device__ __forceinline__ const uint8_t* cslot_wait(const FusedParams& p, const Ctx& c, Cons& w)
+{
+    const uint32_t s = w.it % (uint32_t)p.nslot;
+    mwait(&c.hd->full[s], (w.it / (uint32_t)p.nslot) & 1u, p.status, 51, c.dead);
+    return c.ring + (size_t)s * p.slot_bytes;
+}
+
+__device__ __forceinline__ void cslot_free(const FusedParams& p, const Ctx& c, Cons& w)
+{
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(&c.hd->empty[w.it % (uint32_t)p.nslot]);
+    w.it++;
+}
+
+// router items of this CTA: partial logits in double over the item's columns
+__device__ __forceinline__ void router_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
+                                               const float* xin)
+{
+    const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
+    const int T = p.T, E = p.E, H = p.H, RKc = p.RKc, RC = p.RC, lane = c.lane;
+    const uint8_t* sb = cslot_wait(p, c, w);
+    int mine = 0;
+    constexpr int U = 4;   // float4 per lane per pass
+    for (int i = c.ri0 + c.warp; i < c.ri1; i += NCW) {
+        const int e = i / RC, cc = i - e * RC;
+        const float4* wr = reinterpret_cast<const float4*>(sb + (size_t)(i - c.ri0) * RKc * 4);
+#pragma unroll 1
+        for (int t = 0; t < T; t++) {
+            const double r = c.hd->rnorm[t];
+            double acc = 0.0;
+            for (int u0 = 0; u0 < RKc / 4; u0 += 32 * U) {
+                float4 xv[U];
+#pragma unroll
+                for (int j = 0; j < U; j++) {
+                    const int u = u0 + 32 * j + lane;
+                    xv[j] = u < RKc / 4 ? __ldcg(reinterpret_cast<const float4*>(xin + (size_t)t * H + cc * RKc + 4 * u))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < U; j++) {
+                    const int u = u0 + 32 * j + lane;
+                    if (u < RKc / 4) {
+                        const float4 wv = wr[u];
+                        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+                        if (gamma) gm = __ldg(reinterpret_cast<const float4*>(gamma + cc * RKc + 4 * u));
+                        const float4 x = xv[j];
+                        // n = float(x * r * gamma): exactly x for a plain input
+                        acc = fma((double)(float)((double)x.x * r * (double)gm.x), (double)wv.x, acc);
+                        acc = fma((double)(float)((double)x.y * r * (double)gm.y), (double)wv.y, acc);
+                        acc = fma((double)(float)((double)x.z * r * (double)gm.z), (double)wv.z, acc);
+                        acc = fma((double)(float)((double)x.w * r * (double)gm.w), (double)wv.w, acc);
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) p.rpart[((size_t)t * E + e) * RC + cc] = acc;
+        }
+        mine++;
+    }
+    cslot_free(p, c, w);
+    if (lane == 0 && mine > 0) red_release_add(&layer_cnt(p, l)[0], (uint32_t)mine);
+}
+
+// RMSNorm factors (stacks; 1 otherwise) and the per-token activation scale of the layer
+// input; every CTA sums in the same order, so all CTAs agree bit for bit
+__device__ __forceinline__ void input_scales(const FusedParams& p, const Ctx& c, int l, const float* xin)
+{
+    const int T = p.T, H = p.H, tid = c.tid, lane = c.lane, warp = c.warp;
+    const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
+    Head& hd = *c.hd;
+    constexpr int U = 16;   // values per thread per pass (H <= 6144 in one pass)
+    if (p.norm) {
+#pragma unroll 1
+        for (int t = 0; t < T; t++) {
+            double sq = 0.0;
+            for (int c0 = 0; c0 < H; c0 += NCT * U) {
+                float xv[U];
+#pragma unroll
+                for (int j = 0; j < U; j++) {
+                    const int cc = c0 + NCT * j + tid;
+                    xv[j] = cc < H ? __ldcg(xin + (size_t)t * H + cc) : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < U; j++) sq = fma((double)xv[j], (double)xv[j], sq);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == 0) hd.rsq[warp][t] = sq;
+        }
+        named_bar(5, NCT);
+        if (tid < T) {
+            double sq = 0.0;
+            for (int w = 0; w < NCW; w++) sq += hd.rsq[w][tid];
+            hd.rnorm[tid] = 1.0 / sqrt(sq / (double)H + p.eps);
+        }
+        named_bar(5, NCT);
+    }
+#pragma unroll 1
+    for (int t = 0; t < T; t++) {
+        float mx = 0.0f;
+        const double r = p.norm ? hd.rnorm[t] : 1.0;
+        for (int c0 = 0; c0 < H; c0 += NCT * U) {
+            float xv[U];
+#pragma unroll
+            for (int j = 0; j < U; j++) {
+                const int cc = c0 + NCT * j + tid;
+                xv[j] = cc < H ? __ldcg(xin + (size_t)t * H + cc) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < U; j++) {
+                const int cc = c0 + NCT * j + tid;
+                const double gm = (gamma && cc < H) ? (double)__ldg(gamma + cc) : 1.0;
+                mx = fmaxf(mx, fabsf((float)((double)xv[j] * r * gm)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) hd.amax[warp][t] = mx;
+    }
+    named_bar(5, NCT);
+    if (tid < T) {
+        float mx = 0.0f;
+        for (int w = 0; w < NCW; w++) mx = fmaxf(mx, hd.amax[w][tid]);
+        hd.xinv[tid] = mx > 0.0f ? 126.0f / mx : 0.0f;
+        hd.xfac[tid] = mx * (1.0f / 126.0f);
+    }
+    named_bar(5, NCT);
+}
+
+template <int NTM, int GPWG, bool PAIR>
+__device__ __forceinline__ void build_x_operand(const FusedParams& p, const Ctx& c, Cons& w, int l,
+                                                const float* xin, uint32_t (&Bx)[GPWG][NTM][4],
+                                                float (&fdummy)[GPWG][NTM])
+{
+    const int T = p.T, H = p.H;
+    const Head& hd = *c.hd;
+    const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
+    if constexpr (PAIR) {
+        build_x_pairs<GPWG, NTM>(xin, hd.xinv[0], hd.rnorm[0], gamma, w.gbase_g, w.gpw_g, w.sc, c.lane, Bx);
+    } else {
+#pragma unroll
+        for (int q = 0; q < NTM; q++) {
+            const int t0 = 2 * q, t1 = 2 * q + 1;
+            const bool p0 = t0 < T, p1 = t1 < T;
+            const float* row0 = xin + (size_t)(p0 ? t0 : 0) * H;
+            const float* row1 = xin + (size_t)(p1 ? t1 : 0) * H;
+            build_tile<GPWG, NTM, false>(row0, row1, p0, p1, p0 ? hd.xinv[t0] : 0.0f, p1 ? hd.xinv[t1] : 0.0f,
+                                         hd.rnorm[p0 ? t0 : 0], hd.rnorm[p1 ? t1 : 0], gamma, 0u,
+                                         w.gbase_g, w.gpw_g, q, w.sc, c.lane, Bx, fdummy, p.status, c.dead);
+        }
+    }
+}
+
+// one gate/up stage (stage st of segment s, tokens sg): SwiGLU rows into h
+template <int NTM, int GPWG, bool PAIR>
+__device__ __forceinline__ void gu_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
+                                           const Seg& sg, int st,
+                                           const uint32_t (&Bx)[GPWG][NTM][4],
+                                           const float (&fdummy)[GPWG][NTM])
+{
+    const int T = p.T, H = p.H, I = p.I, lane = c.lane;
+    const uint8_t* sb = cslot_wait(p, c, w);
+    const int i0 = st * 8 * p.NTSg;
+    const int ntl = min(p.NTSg, (I - i0) / 8);
+    const int cr = 2 * ntl;    // rows per chunk
+    uint32_t qmask = 0;
+    for (int m = 0; m < sg.c; m++) qmask |= 1u << (sg.tok[m] >> 1);
+    red_wait_free(*c.hd, w.cs, p.status, c.dead, lane);
+    float* rb = c.red + (size_t)(w.cs % kRedBufs) * p.red_floats;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t rowb = (uint32_t)H / 2, srow = (uint32_t)H / 64;
+    for (int tl = w.g_rs; tl < ntl; tl += p.RSg) {
+        // lane row g: chunk g & 3, row 2 tl + (g >> 2) of the chunk
+        const int lr = 2 * tl + (g >> 2);
+        const uint8_t* ga = sb + (size_t)(g & 3) * p.gu_chunk + (size_t)lr * rowb + (PAIR ? 16 : 8) * t;
+        const uint8_t* ua = ga + (size_t)4 * p.gu_chunk;
+        const int sr = (g & 3) * cr + lr;
+        const __half* gs = reinterpret_cast<const __half*>(sb + p.gu_gsc) + (size_t)sr * srow;
+        const __half* us = reinterpret_cast<const __half*>(sb + p.gu_usc) + (size_t)sr * srow;
+        float* rbt = rb + (size_t)(w.g_kw * p.NTSg + tl) * 16 * T;
+        if constexpr (PAIR) {
+            float acc4[4];
+            tile_dot_pairs<GPWG, NTM, false>(ga, ua, gs, us, w.gbase_g, lane, Bx, fdummy, acc4);
+            tile_partials_pairs(acc4, lane, rbt, c.hd->xfac[0]);
+        } else {
+            float acc[NTM][4];
+            tile_dot<GPWG, NTM, false>(ga, ua, gs, us, w.gbase_g, w.gpw_g, qmask, Bx, fdummy, acc);
+            tile_partials<NTM>(acc, qmask, lane, T, rbt, T, c.hd->xfac);
+        }
+    }
+    cslot_free(p, c, w);
+    red_deliver(*c.hd, w.cs, lane);
+    w.cs++;
+}
+
+// the down stage of segment s (this CTA's output rows), combined into yacc
+template <int NTM, int GPWD, bool PAIR>
+__device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
+                                             const Seg& sg, uint32_t (&Bh)[GPWD][NTM][4],
+                                             float (&fh)[GPWD][NTM])
+{
+    const int T = p.T, I = p.I, lane = c.lane;
+    const int cn = sg.c;
+    const uint32_t ep = h_epoch(c, l);
+    const uint2* hb = reinterpret_cast<const uint2*>(p.h);
+    if constexpr (PAIR) {
+        // the segment's h digits once per CTA (double-buffered), then each warp's operand
+        uint8_t* hd0 = reinterpret_cast<uint8_t*>(c.hd) + p.off_hdig + (size_t)(w.ds & 1) * p.hdig_bytes;
+        uint32_t* dig = reinterpret_cast<uint32_t*>(hd0);
+        float* facs = reinterpret_cast<float*>(hd0 + 3 * I);
+        digitize_h_row(hb + (size_t)sg.base * I, ep, I, c.warp, lane, w.sc, dig, facs, p.status, c.dead);
+        named_bar(6, NCT);
+        gather_h_pairs<GPWD, NTM>(dig, facs, I, w.gbase_d, lane, Bh, fh);
+        w.ds++;
+    } else {
+#pragma unroll
+        for (int q = 0; q < NTM; q++) {
+            const int m0 = 2 * q, m1 = 2 * q + 1;
+            const bool p0 = m0 < cn, p1 = m1 < cn;
+            const uint2* row0 = hb + (size_t)(sg.base + (p0 ? m0 : 0)) * I;
+            const uint2* row1 = hb + (size_t)(sg.base + (p1 ? m1 : 0)) * I;
+            build_tile<GPWD, NTM, true>(row0, row1, p0, p1, 0.f, 0.f, 1.0, 1.0, nullptr, ep,
+                                        w.gbase_d, w.gpw_d, q, w.sc, lane, Bh, fh, p.status, c.dead);
+        }
+    }
+    const uint32_t qmask = (1u << ((cn + 1) >> 1)) - 1u;
+    const uint8_t* sb = cslot_wait(p, c, w);
+    red_wait_free(*c.hd, w.cs, p.status, c.dead, lane);
+    float* rb = c.red + (size_t)(w.cs % kRedBufs) * p.red_floats;
+    const uint32_t delta = (uint32_t)(((uint64_t)c.r0 * (I / 32)) & 15ull);
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t rowb = (uint32_t)I / 2, srow = (uint32_t)I / 64;
+    const __half* scb = reinterpret_cast<const __half*>(sb + p.d_sc_off + delta);
+    const int ntdm = p.ntdm;
+    for (int tl = w.d_rs; tl < c.ntd; tl += p.RSd) {
+        // MMA row m: chunk m & 3, row 4 tl + (m >> 2) of the chunk (rows g and g + 8)
+        const int q = g & 3, la = 4 * tl + (g >> 2), lb = la + 2;
+        const uint8_t* ra = sb + (size_t)q * p.d_chunk + (size_t)la * rowb + (PAIR ? 16 : 8) * t;
+        const uint8_t* rbp = sb + (size_t)q * p.d_chunk + (size_t)lb * rowb + (PAIR ? 16 : 8) * t;
+        const __half* sa = scb + (size_t)(dcs(c, q) + la) * srow;
+        const __half* sbh = scb + (size_t)(dcs(c, q) + lb) * srow;
+        float* rbt = rb + (size_t)(w.d_kw * ntdm + tl) * 16 * T;
+        if constexpr (PAIR) {
+            float acc4[4];
+            tile_dot_pairs<GPWD, NTM, true>(ra, rbp, sa, sbh, w.gbase_d, lane, Bh, fh, acc4);
+            tile_partials_pairs(acc4, lane, rbt, 1.0f);
+        } else {
+            float acc[NTM][4];
+            tile_dot<GPWD, NTM, true>(ra, rbp, sa, sbh, w.gbase_d, w.gpw_d, qmask, Bh, fh, acc);
+            tile_partials<NTM>(acc, qmask, lane, cn, rbt, T, nullptr);
+        }
+    }
+    cslot_free(p, c, w);
+    red_deliver(*c.hd, w.cs, lane);
+    w.cs++;
+}
+
+// ----------------------------- reducer warp ---------------------------------------------
+// Sums of one gate/up stage (stage st of segment sg): four lanes per (row, token) over the
+// K-split warps' partials, SwiGLU, h stored as (value, epoch).
+__device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, uint32_t cs, const Seg& sg,
+                                          int st, uint32_t ep)
+{
+    const int T = p.T, I = p.I, lane = c.lane;
+    const float* rb = c.red + (size_t)(cs % kRedBufs) * p.red_floats;
+    const int i0 = st * 8 * p.NTSg;
+    const int ntl = min(p.NTSg, (I - i0) / 8);
+    const int cr = 2 * ntl;
+    uint2* hb = reinterpret_cast<uint2*>(p.h);
+    const int ntask = ntl * 8 * sg.c, part = lane & 3;
+    for (int t0 = 0; t0 < ntask; t0 += 8) {
+        const int task = t0 + (lane >> 2);
+        const bool valid = task < ntask;
+        const int m = valid ? task % sg.c : 0, rr = valid ? task / sg.c : 0;
+        const int tl = rr >> 3, r = rr & 7;
+        const int tok = sg.tok[m];
+        float gsum = 0.0f, usum = 0.0f;
+        if (valid)
+            for (int kw = part; kw < p.KWg; kw += 4) {
+                const float* q = rb + (size_t)(kw * p.NTSg + tl) * 16 * T;
+                gsum += q[r * T + tok];
+                usum += q[(8 + r) * T + tok];
+            }
+        gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
+        usum += __shfl_xor_sync(0xffffffffu, usum, 1);
+        gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
+        usum += __shfl_xor_sync(0xffffffffu, usum, 2);
+        if (valid && part == 0) {
+            const float hv = gsum / (1.0f + expf(-gsum)) * usum;
+            const int row = i0 + (r & 3) * cr + 2 * tl + (r >> 2);
+            hb[(size_t)(sg.base + m) * I + row] = make_uint2(__float_as_uint(hv), ep);
+        }
+    }
+}
+
+// Sums of one down stage (segment sg, the CTA's rows): routing-weighted combine into yacc.
+__device__ __forceinline__ void reduce_down(const FusedParams& p, const Ctx& c, uint32_t cs, const Seg& sg)
+{
+    const int T = p.T, lane = c.lane, cn = sg.c, ntdm = p.ntdm;
+    const float* rb = c.red + (size_t)(cs % kRedBufs) * p.red_floats;
+    const int ntask = c.ntd * 16 * cn, part = lane & 3;
+    for (int t0 = 0; t0 < ntask; t0 += 8) {
+        const int task = t0 + (lane >> 2);
+        const int m = task % cn, rr = task / cn;
+        const int tl = rr >> 4, mm = rr & 15;
+        const int q = mm & 3, lrow = 4 * tl + (mm >> 2);
+        const bool valid = task < ntask && lrow < dcs(c, q + 1) - dcs(c, q);
+        float sum = 0.0f;
+        if (valid)
+            for (int kw = part; kw < p.KWd; kw += 4) sum += rb[((size_t)(kw * ntdm + tl) * 16 + mm) * T + m];
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (valid && part == 0) {
+            float* ya = c.yacc + (dcs(c, q) + lrow) * T + sg.tok[m];
+            *ya = *ya + sg.wt[m] * sum;
+        }
+    }
+}
+
+// The reducer follows the consumers' sequence of reduction stages.
+__device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c, uint32_t gen)
+{
+    const int T = p.T, k = p.k, ns = p.n_shared, lane = c.lane;
+    Seg sh;
+    sh.c = T;
+    sh.base = T * k;
+    sh.tok = c.hd->sh_tok;
+    sh.wt = c.hd->sh_wt;
+    uint32_t cs = 0;
+    auto take = [&]() {
+        mwait(&c.hd->red_full[cs % kRedBufs], (cs / kRedBufs) & 1u, p.status, 59, c.dead);
+    };
+    auto give = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.hd->red_empty[cs % kRedBufs]);
+        cs++;
+    };
+    for (int l = 0; l < p.L; l++) {
+        const uint32_t ep = gen * 32u + (uint32_t)l + 1u;
+        int gi = c.b;
+        if (ns) {
+            for (; gi < p.SPS; gi += c.G) {
+                take();
+                reduce_gu(p, c, cs, sh, gi, ep);
+                give();
+            }
+            if (c.nrows > 0) {
+                take();
+                reduce_down(p, c, cs, sh);
+                give();
+            }
+        }
+        mwait(&c.hd->route_bar, (uint32_t)l & 1u, p.status, 60, c.dead);
+        const Table tb = layer_table(c, l);
+        const int nseg = tb.hdr[0];
+        while (gi < ns * p.SPS) gi += c.G;
+        for (; gi < nseg * p.SPS; gi += c.G) {
+            const int sg = gi / p.SPS;
+            take();
+            reduce_gu(p, c, cs, seg_of(tb, sg), gi - sg * p.SPS, ep);
+            give();
+        }
+        if (c.nrows > 0)
+            for (int sg = ns; sg < nseg; sg++) {
+                take();
+                reduce_down(p, c, cs, seg_of(tb, sg));
+                give();
+            }
+        // the layer's output rows are summed: the consumers write them, then yacc is clear
+        named_bar(7, NCT + 32);
+        named_bar(8, NCT + 32);
+    }
+}
+
+template <int NTM, int GPWG, int GPWD, bool PAIR>
+__device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c)
+{
+    const int T = p.T, H = p.H, k = p.k, ns = p.n_shared;
+    Cons w;
+    w.it = 0;
+    w.cs = 0;
+    w.ds = 0;
+    w.sc = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_scratch) + c.warp * 96;
+    // K split: warp kw of a row slot takes groups [kw n / KW, (kw + 1) n / KW)
+    const int ngg = p.H / 64, ngd = p.I / 64;
+    w.g_rs = c.warp / p.KWg;
+    w.g_kw = c.warp % p.KWg;
+    w.gbase_g = w.g_kw * ngg / p.KWg;
+    w.gpw_g = (w.g_kw + 1) * ngg / p.KWg - w.gbase_g;
+    w.d_rs = c.warp / p.KWd;
+    w.d_kw = c.warp % p.KWd;
+    w.gbase_d = w.d_kw * ngd / p.KWd;
+    w.gpw_d = (w.d_kw + 1) * ngd / p.KWd - w.gbase_d;
+    uint32_t Bx[GPWG][NTM][4];
+    float fdummy[GPWG][NTM];
+    uint32_t Bh[GPWD][NTM][4];
+    float fh[GPWD][NTM];
+#pragma unroll
+    for (int gi = 0; gi < GPWG; gi++)
+#pragma unroll
+        for (int q = 0; q < NTM; q++) fdummy[gi][q] = 0.0f;
+    Seg sh;
+    sh.c = T;
+    sh.base = T * k;
+    sh.tok = c.hd->sh_tok;
+    sh.wt = c.hd->sh_wt;
+
+    for (int l = 0; l < p.L; l++) {
+        uint32_t* lc = layer_cnt(p, l);
+        const float* xin = l == 0 ? p.x : p.xbuf + (size_t)((l - 1) & 1) * T * H;
+        float* yout = l == p.L - 1 ? p.y : p.xbuf + (size_t)(l & 1) * T * H;
+        const float* res = p.norm ? xin : p.residual;
+        if (l > 0) {
+            if (c.lane == 0) gwait(&layer_cnt(p, l - 1)[1], (uint32_t)c.G, p.status, 52, c.dead);
+            __syncwarp();
+        }
+        // the router needs only the RMSNorm factors (1 for a plain input), so for a plain
+        // input it runs first and the routing is decided while the scales are formed
+        if (!p.norm && c.ri1 > c.ri0) router_consume(p, c, w, l, xin);
+        input_scales(p, c, l, xin);
+        if (p.norm && c.ri1 > c.ri0) router_consume(p, c, w, l, xin);
+        // stages in the control warp's order; one code path per kind of step
+        //   phase 0: x operand, 1: shared gate/up, 2: shared down, 3: x operand again,
+        //   4: routing, 5: routed gate/up, 6: routed down
+        Table tb;
+        int nseg = 0, phase = 0, gi = c.b, sd = ns;
+        while (true) {
+            int kind = -1, seg = 0, stage = 0;   // 0: x operand, 1: gate/up, 2: down
+            if (phase == 0) {
+                kind = 0;
+                phase = 1;
+            } else if (phase == 1) {
+                if (ns && gi < p.SPS) {
+                    kind = 1;
+                    seg = 0;
+                    stage = gi;
+                    gi += c.G;
+                } else {
+                    phase = 2;
+                    continue;
+                }
+            } else if (phase == 2) {
+                phase = 4;
+                if (ns && c.nrows > 0) {
+                    kind = 2;
+                    seg = 0;
+                    phase = 3;
+                } else {
+                    continue;
+                }
+            } else if (phase == 3) {
+                kind = 0;
+                phase = 4;
+            } else if (phase == 4) {
+                mwait(&c.hd->route_bar, (uint32_t)l & 1u, p.status, 55, c.dead);
+                tb = layer_table(c, l);
+                nseg = tb.hdr[0];
+                while (gi < ns * p.SPS) gi += c.G;
+                phase = 5;
+                continue;
+            } else if (phase == 5) {
+                if (gi < nseg * p.SPS) {
+                    kind = 1;
+                    seg = gi / p.SPS;
+                    stage = gi - seg * p.SPS;
+                    gi += c.G;
+                } else {
+                    phase = 6;
+                    continue;
+                }
+            } else {
+                if (c.nrows > 0 && sd < nseg) {
+                    kind = 2;
+                    seg = sd++;
+                } else {
+                    break;
+                }
+            }
+            if (kind == 0) {
+                build_x_operand<NTM, GPWG, PAIR>(p, c, w, l, xin, Bx, fdummy);
+            } else {
+                const Seg sg = seg < ns ? sh : seg_of(tb, seg);
+                if (kind == 1) {
+                    gu_consume<NTM, GPWG, PAIR>(p, c, w, l, sg, stage, Bx, fdummy);
+                } else if constexpr (GPWG == GPWD) {
+                    // the h operand takes the x operand's registers (x is rebuilt after the
+                    // shared expert's down stage and not needed after the routed ones)
+                    down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bx, fdummy);
+                } else {
+                    down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bh, fh);
+                }
+            }
+        }
+        // ---- this CTA's rows of the layer output (once the reducer has summed them all)
+        named_bar(7, NCT + 32);
+        for (int i = c.tid; i < c.nrows * T; i += NCT) {
+            const int rr = i / T, t = i - rr * T;
+            const size_t o = (size_t)t * H + c.r0 + rr;
+            const float base = res ? __ldcg(res + o) : 0.0f;
+            yout[o] = base + c.yacc[i];
+            c.yacc[i] = 0.0f;
+        }
+        named_bar(8, NCT + 32);
+        if (c.tid == 0) {
+            __threadfence();
+            red_release_add(&lc[1], 1u);
+        }
+    }
+}
+
+template <int NTM, int GPWG, int GPWD, bool PAIR>
+__global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constant__ FusedParams p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    Ctx c;
+    c.hd = reinterpret_cast<Head*>(smem);
+    c.dead = &c.hd->dead;
+    c.ring = smem + p.off_ring;
+    c.red = reinterpret_cast<float*>(smem + p.off_red);
+    c.yacc = reinterpret_cast<float*>(smem + p.off_yacc);
+    c.rt_base = smem + sizeof(Head);
+    c.S = 1 + p.T * p.k;
+    c.tbytes = table_bytes(c.S);
+    c.tid = threadIdx.x;
+    c.warp = c.tid >> 5;
+    c.lane = c.tid & 31;
+    c.b = blockIdx.x;
+    c.G = gridDim.x;
+    c.r0 = (int)((int64_t)p.H * c.b / c.G);
+    c.r1 = (int)((int64_t)p.H * (c.b + 1) / c.G);
+    c.nrows = c.r1 - c.r0;
+    c.ntd = (((c.nrows + 3) >> 2) + 3) >> 2;
+    c.n_ritems = p.E * p.RC;
+    c.ri0 = p.route ? (int)((int64_t)c.n_ritems * c.b / c.G) : 0;
+    c.ri1 = p.route ? (int)((int64_t)c.n_ritems * (c.b + 1) / c.G) : 0;
+    c.bo = blob_off(p.H, p.I);
+
+    pdl_launch_dependents();
+    if (c.tid == 0) {
+        for (int s = 0; s < p.nslot; s++) {
+            mbar_init(&c.hd->full[s], 1);
+            mbar_init(&c.hd->empty[s], NCW);
+        }
+        mbar_init(&c.hd->route_bar, 1);
+        c.hd->dead = 0;
+        for (int b2 = 0; b2 < kRedBufs; b2++) {
+            mbar_init(&c.hd->red_full[b2], NCW);
+            mbar_init(&c.hd->red_empty[b2], 1);
+        }
+        for (int m = 0; m < kFusedMaxT; m++) {
+            c.hd->sh_tok[m] = m;
+            c.hd->sh_wt[m] = 1.0f;
+            c.hd->rnorm[m] = 1.0;
+        }
+        fence_barrier_init();
+    }
+    for (int i = c.tid; i < p.rows_max * p.T; i += NTHR) c.yacc[i] = 0.0f;
+    __syncthreads();
+
+    if (c.warp == NCW) {
+        control_warp(p, c);
+    } else if (c.warp == NCW + 1) {
+        pdl_wait();
+        reducer_warp(p, c, __ldcg(p.gen));
+    } else {
+        pdl_wait();
+        if (c.tid == 0) c.hd->gen = __ldcg(p.gen);   // published by the first named barrier
+        consumer_warp<NTM, GPWG, GPWD, PAIR>(p, c);
+    }
+
+    // ---- exit: the last CTA returns the counters to zero and advances the generation
+    __syncthreads();
+    if (c.tid == 0) {
+        __threadfence();
+        const uint32_t prev = atomicAdd(&p.cnt[0], 1u);
+        if (prev == (uint32_t)c.G - 1u) {
+            __threadfence();
+            for (int i = 1; i < 1 + p.L * kCntPerLayer; i++) p.cnt[i] = 0u;
+            *p.gen = c.hd->gen + 1u;
+            __threadfence();
+            p.cnt[0] = 0u;
+        }
+    }
+}
+
+template <int NTM, int GPWG, int GPWD, bool PAIR>
+cudaError_t launch_fused(const FusedParams& p, cudaStream_t s)
+{
+    auto kern = fused_moe_kernel<NTM, GPWG, GPWD, PAIR>;
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || set_bytes[dev] < (int)p.smem) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) set_bytes[dev] = (int)p.smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(NTHR);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+inline uint32_t up128(uint32_t v) { return (v + 127u) / 128u * 128u; }
+
+// K-split of a matrix with n 64-column groups over the consumer warps: the largest divisor
+// of the warp count not above n (the remaining warps take further row tiles).
+inline int kw_for(int n)
+{
+    const int cand[6] = {12, 6, 4, 3, 2, 1};
+    for (int i = 0; i < 6; i++)
+        if (cand[i] <= n) return cand[i];
+    return 1;
+}
+
+// Stride of the four row chunks of a stage: at least `bytes`, and 32 bytes more than a
+// multiple of 128, so the same row of the four chunks falls on four different bank groups.
+inline uint32_t chunk_stride(uint32_t bytes) { return (bytes + 95u) / 128u * 128u + 32u; }
+inline uint32_t chunk_stride64(uint32_t bytes) { return (bytes + 63u) / 128u * 128u + 64u; }
+
+// Pair-mode K split: the largest divisor of the warp count giving every warp exactly 8 (or
+// else 4) of the n groups; 0 if none.
+inline int kw_pair(int n)
+{
+    const int cand[6] = {12, 6, 4, 3, 2, 1};
+    for (int per : {8, 4})
+        for (int i = 0; i < 6; i++)
+            if (n == cand[i] * per) return cand[i];
+    return 0;
+}
+
+constexpr int kGpwMax = 8;
+
+}  // namespace
+
+bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
+{
+    const int H = p.H, I = p.I, E = p.E, T = p.T;
+    if (T < 1 || T > kFusedMaxT || p.L < 1 || p.L > kFusedMaxLayers) return false;
+    if (p.k < 1 || p.k > kFusedMaxK || p.k > E || E > 1024) return false;
+    if (H % 128 || I % 64 || H < 128 || I < 64) return false;
+    if (p.L > 1 && !p.norm) return false;
+    p.NT = (T + 1) / 2;
+    const int G = num_sms;
+    p.grid = G;
+    // gate/up: K = H; down: K = I
+    const int ngg = H / 64, ngd = I / 64;
+    p.KWg = kw_for(ngg);
+    p.RSg = NCW / p.KWg;
+    p.GPWg = (ngg + p.KWg - 1) / p.KWg;   // groups of the widest warp
+    p.KWd = kw_for(ngd);
+    p.RSd = NCW / p.KWd;
+    p.GPWd = (ngd + p.KWd - 1) / p.KWd;
+    if (p.GPWg > kGpwMax || p.GPWd > kGpwMax) return false;
+    // gate/up stage: NTSg row tiles, about 32 KB or more, dividing the I / 8 tiles of a
+    // segment when that is possible
+    const uint32_t tile_all = 16u * (uint32_t)H / 2u + 16u * (uint32_t)H / 32u;
+    int nts = (int)(32768u / tile_all);
+    if (nts < 1) nts = 1;
+    while (nts > 1 && 8 * nts > I) nts--;
+    for (int n = nts; n >= 1; n--)
+        if ((I / 8) % n == 0) {
+            if (n * 2 >= nts) nts = n;
+            break;
+        }
+    p.NTSg = nts;
+    p.SPS = (I + 8 * nts - 1) / (8 * nts);
+    // one token: both matrices in group pairs when each splits into warp shares of exactly 4
+    // or 8 aligned groups; the 16-byte row reads need the chunks 64 bytes (mod 128) apart
+    p.pair = 0;
+    if (T == 1 && H % 512 == 0 && I % 512 == 0) {
+        const int kg = kw_pair(ngg), kd = kw_pair(ngd);
+        if (kg && kd) {
+            p.pair = 1;
+            p.KWg = kg;
+            p.RSg = NCW / kg;
+            p.GPWg = ngg / kg;
+            p.KWd = kd;
+            p.RSd = NCW / kd;
+            p.GPWd = ngd / kd;
+            // the stage's row tiles are a multiple of the row slots
+            int n2 = (int)(32768u / (16u * (uint32_t)H / 2u + 16u * (uint32_t)H / 32u));
+            if (n2 < 1) n2 = 1;
+            n2 = (n2 + p.RSg - 1) / p.RSg * p.RSg;
+            while (n2 > p.RSg && ((I / 8) % n2 != 0 || 8 * n2 > I)) n2 -= p.RSg;
+            if ((I / 8) % n2 == 0 && 8 * n2 <= I) {
+                nts = n2;
+                p.NTSg = nts;
+                p.SPS = (I + 8 * nts - 1) / (8 * nts);
+            }
+        }
+    }
+    p.gu_chunk = p.pair ? chunk_stride64(2u * nts * (uint32_t)H / 2u)
+                        : chunk_stride(2u * nts * (uint32_t)H / 2u);
+    p.gu_gsc = 8u * p.gu_chunk;
+    p.gu_usc = p.gu_gsc + 8u * nts * (uint32_t)H / 32u;
+    const uint32_t gu_stage = p.gu_usc + 8u * nts * (uint32_t)H / 32u;
+    // down stage: the CTA's rows in four chunks, tiles of four rows per chunk
+    p.rows_max = (H + G - 1) / G;
+    p.ntdm = (((p.rows_max + 3) / 4) + 3) / 4;
+    p.d_chunk = p.pair ? chunk_stride64(4u * p.ntdm * (uint32_t)I / 2u)
+                       : chunk_stride(4u * p.ntdm * (uint32_t)I / 2u);
+    p.d_sc_off = 4u * p.d_chunk;
+    const uint32_t d_stage = p.d_sc_off + (uint32_t)(p.rows_max + 16) * (uint32_t)I / 32u + 32u;
+    // router: column chunks so that every CTA gets about one item per consumer warp
+    p.RC = 1;
+    while (p.RC < 8 && E * p.RC * 2 <= NCW * G && (H / (2 * p.RC)) % 128 == 0) p.RC *= 2;
+    p.RKc = H / p.RC;
+    const int items_max = (E * p.RC + G - 1) / G;
+    const uint32_t r_stage = (uint32_t)items_max * (uint32_t)p.RKc * 4u;
+    uint32_t slot = gu_stage > d_stage ? gu_stage : d_stage;
+    if (r_stage > slot) slot = r_stage;
+    p.slot_bytes = up128(slot);
+    // fixed shared memory: head, two routing tables, partial sums, y rows, scratch
+    const int S = 1 + T * p.k;
+    uint32_t off = up128((uint32_t)sizeof(Head) + 2u * table_bytes(S));
+    p.off_red = off;
+    const uint32_t red_g = (uint32_t)p.KWg * p.NTSg * 16u * T;
+    const uint32_t red_d = (uint32_t)p.KWd * p.ntdm * 16u * T;
+    p.red_floats = red_g > red_d ? red_g : red_d;
+    off = up128(off + (uint32_t)kRedBufs * p.red_floats * 4u);
+    p.off_yacc = off;
+    off = up128(off + (uint32_t)p.rows_max * T * 4u);
+    p.hdig_bytes = p.pair ? (uint32_t)(3 * I + 4 * (I / 64)) : 0u;
+    p.off_hdig = off;
+    off = up128(off + 2u * p.hdig_bytes);
+    p.off_scratch = off;
+    // consumer digit scratch (96 words per warp), then the control warp's logits,
+    // selections, weights and bitmaps
+    off = up128(off + NCW * 96u * 4u + (uint32_t)(T * E) * 4u + 2u * (uint32_t)(T * p.k) * 4u +
+                kFusedMaxT * 32u * 4u);
+    p.off_ring = off;
+    if (off + 2u * p.slot_bytes > smem_limit) return false;
+    int nslot = (int)((smem_limit - off) / p.slot_bytes);
+    if (nslot > kMaxSlots) nslot = kMaxSlots;
+    p.nslot = nslot;
+    p.smem = off + (size_t)nslot * p.slot_bytes;
+    return true;
+}
+
+// Kernel variants by MMA column tiles and the widest warp's group count (registers hold
+// one B operand per group): gate/up up to 4 or 8 groups, down up to 3 or 8.
+template <int NTM, bool PAIR>
+static cudaError_t launch_nt(const FusedParams& p, cudaStream_t s)
+{
+    if (p.GPWg <= 4)
+        return p.GPWd <= 3 ? launch_fused<NTM, 4, 3, PAIR>(p, s) : launch_fused<NTM, 4, 8, PAIR>(p, s);
+    return p.GPWd <= 3 ? launch_fused<NTM, 8, 3, PAIR>(p, s) : launch_fused<NTM, 8, 8, PAIR>(p, s);
+}
+
+// Pair mode: the warps' group counts exactly (4 or 8 for each matrix).
+cudaError_t launch_pair(const FusedParams& p, cudaStream_t s)
+{
+    if (p.GPWg == 8) return p.GPWd == 8 ? launch_fused<1, 8, 8, true>(p, s) : launch_fused<1, 8, 4, true>(p, s);
+    return p.GPWd == 8 ? launch_fused<1, 4, 8, true>(p, s) : launch_fused<1, 4, 4, true>(p, s);
+}
+
+cudaError_t fused_launch(const FusedParams& p, cudaStream_t s)
+{
+    if (p.NT == 2) return launch_nt<2, false>(p, s);
+    return p.pair ? launch_pair(p, s) : launch_nt<1, false>(p, s);
+}
+
+}  // namespace coli

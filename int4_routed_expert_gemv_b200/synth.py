@@ -218,6 +218,9 @@ WORKLOADS = {
         Workload("glm52_stack16_h6144_i2048_e256_k8_t1", GLM, 1, seed=3, x_variant=0,
                  layers=16,
                  description="16 GLM-5.2-shaped layers, x <- x + MoE(RMSNorm(x)), 1 token"),
+        Workload("moe_h1024_i512_e64_k4_stack16_t1", SMALL, 1, seed=3, x_variant=0, layers=16,
+                 description="16 hidden-1024 layers (64 experts of intermediate 512, top-4 + 1 "
+                             "shared each), x <- x + MoE(RMSNorm(x)), 1 token"),
         Workload("moe_h1024_i512_e64_k4_t2048_bf16_zipf", SMALL, 2048, seed=0, x_variant=2,
                  zipf=True, x_dtype="bf16",
                  description="prefill-like 2048 bf16 tokens through the hidden-1024 layer, "

@@ -86,3 +86,18 @@ def test_glm_stack16_decode(colimoe):
     # the oracle's own chain amplifies a 2^-24 input change only to ~4e-7 over 16 layers,
     # so the free-running stack is held to the per-layer bar as well
     assert_y_close(x.cpu().numpy(), xs_o[-1])
+
+    # the same 16 layers as one resident launch (coli_moe_stack)
+    ws = torch.zeros(B.coli_moe_workspace_bytes(dims, T), dtype=torch.uint8, device="cuda")
+    B.check(B.coli_moe_workspace_init(ws))
+    y = torch.empty(T, s.hidden, device="cuda")
+    idx_all = torch.full((L, T, s.top_k), -1, dtype=torch.int32, device="cuda")
+    B.check(B.coli_moe_stack(dims, [lay[4] for lay in layers], [gamma] * L, 1e-5,
+                             torch.from_numpy(x0).cuda(), T, idx_all, y, ws), "coli_moe_stack")
+    for l in range(L):
+        assert np.array_equal(idx_all[l].cpu().numpy(), idx_o[l]), f"stack launch layer {l}: experts differ"
+    rel, mx = y_errors(y.cpu().numpy(), xs_o[-1])
+    print(f"one-launch stack final x: rel L2 {rel:.2e}  max/rms {mx:.2e}")
+    assert_y_close(y.cpu().numpy(), xs_o[-1])
+    st, bits = B.coli_moe_read_status(ws)
+    assert st == B.COLI_OK and bits == 0
