@@ -53,7 +53,7 @@ WsLayout ws_layout(const coli_moe_dims* d, int64_t T)
     // outputs of a stack launch, and the outputs of stack launches but the last
     const int64_t Tf = T < kFusedMaxT ? T : kFusedMaxT;
     L.rpart = off = up(off, kAlign);
-    off += (size_t)Tf * d->n_experts * (d->hidden / 128 > 0 ? d->hidden / 128 : 1) * sizeof(double);
+    off += (size_t)Tf * d->n_experts * (d->hidden / 128 > 0 ? d->hidden / 128 : 1) * 16;
     L.hf = off = up(off, kAlign);   // SwiGLU activations as (value, epoch) pairs
     off += (size_t)Tf * (d->top_k + d->n_shared) * d->inter * 8;
     L.xbuf = off = up(off, kAlign);
@@ -185,7 +185,7 @@ bool fused_setup(FusedParams& f, const coli_moe_dims* d, int32_t T, int L, void*
     f.status = &hdr->status;
     f.gen = &hdr->launch_gen;
     f.cnt = reinterpret_cast<uint32_t*>(base + W.cnt);
-    f.rpart = reinterpret_cast<double*>(base + W.rpart);
+    f.rpart = reinterpret_cast<uint4*>(base + W.rpart);
     f.h = reinterpret_cast<uint2*>(base + W.hf);
     f.xbuf = reinterpret_cast<float*>(base + W.xbuf);
     return true;

@@ -132,6 +132,19 @@ __device__ __forceinline__ void bulk_g2s_hint(void* smem_dst, const void* gsrc, 
         : "memory");
 }
 
+// Asynchronous 16-byte copy global -> shared through L2 (cp.async.cg); groups of them are
+// committed and awaited per thread.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Programmatic dependent launch.  launch_dependents lets the next kernel of the stream
 // (launched with programmatic stream serialization) be scheduled before this one ends;
 // wait blocks until the kernels this one depends on have completed and their memory is

@@ -513,10 +513,10 @@ __device__ __forceinline__ void tile_partials(const float (&acc)[NTM][4], uint32
 // Operand of pair P of the warp's groups for the layer input (token 0): Bp[pair][8] in the
 // register array B[2P + (r >> 2)][0][r & 3], r = 0..7 (MMA j uses registers 2j, 2j + 1).
 template <int GPWM, int NTM>
-__device__ __forceinline__ void build_x_pairs(const float* row, float inv, double rn,
-                                              const float* gamma, int gbase, int gpw, uint32_t* sc,
+__device__ __forceinline__ void build_x_pairs(const float* row, float inv, int gbase, int gpw, uint32_t* sc,
                                               int lane, uint32_t (&B)[GPWM][NTM][4])
 {
+    // row: the normalised input in shared memory
     constexpr int NP = GPWM / 2;
     const int n = lane >> 2, tq = lane & 3, plane = n & 3;
     const int pl = plane < 3 ? plane : 0;
@@ -524,20 +524,8 @@ __device__ __forceinline__ void build_x_pairs(const float* row, float inv, doubl
     float4 v[NP];
 #pragma unroll
     for (int pi = 0; pi < NP; pi++)
-        v[pi] = 2 * pi < gpw ? __ldcg(reinterpret_cast<const float4*>(row + 64 * (gbase + 2 * pi) + 4 * lane))
+        v[pi] = 2 * pi < gpw ? *reinterpret_cast<const float4*>(row + 64 * (gbase + 2 * pi) + 4 * lane)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    // n = float(x * r * gamma); r = 1 and gamma = 1 leave a plain input exactly as it is
-#pragma unroll
-    for (int pi = 0; pi < NP; pi++) {
-        const int c0 = 64 * (gbase + 2 * pi) + 4 * lane;
-        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (gamma && 2 * pi < gpw) gm = __ldg(reinterpret_cast<const float4*>(gamma + c0));
-        float4& x = v[pi];
-        x.x = (float)((double)x.x * rn * (double)gm.x);
-        x.y = (float)((double)x.y * rn * (double)gm.y);
-        x.z = (float)((double)x.z * rn * (double)gm.z);
-        x.w = (float)((double)x.w * rn * (double)gm.w);
-    }
 #pragma unroll
     for (int pi = 0; pi < NP; pi++) {
         digits128_fixed(v[pi], inv, lane, sc);
@@ -622,26 +610,35 @@ __device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, 
 // Digits of one token's h row (I columns), once per CTA: warp w digitizes group pairs w,
 // w + NCW, ... into the compact buffer dig (plane p: I bytes at p * I, column order) and the
 // group factors m / 126 into fac.  (value, epoch) pairs are read until they carry `epoch`.
-__device__ __forceinline__ void digitize_h_row(const uint2* row, uint32_t epoch, int I, int warp, int lane,
-                                               uint32_t* sc, uint32_t* dig, float* fac,
+__device__ __forceinline__ void digitize_h_row(const uint2* staged, const uint2* row, uint32_t epoch, int I,
+                                               int warp, int lane, uint32_t* sc, uint32_t* dig, float* fac,
                                                uint32_t* status, volatile int* dead)
 {
     const int npairs = I / 128;
+#pragma unroll 1
     for (int pp = warp; pp < npairs; pp += NCW) {
-        const uint4* hp = reinterpret_cast<const uint4*>(row + 128 * pp + 4 * lane);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        const long long t0 = clock64();
-        while (true) {
-            const uint4 a = __ldcg(hp), b = __ldcg(hp + 1);
-            const bool ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
-            v = make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x), __uint_as_float(b.z));
-            if (ok) break;
-            if (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
-                if (lane == 0) give_up(status, 56, dead);
-                break;
+        // the staged copy first; where it holds another epoch's values (the copy ran before
+        // the producer's store), poll the row itself
+        const uint4* sp = reinterpret_cast<const uint4*>(staged + 128 * pp + 4 * lane);
+        uint4 a = sp[0], b = sp[1];
+        bool ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
+        if (!ok) {
+            const uint4* hp = reinterpret_cast<const uint4*>(row + 128 * pp + 4 * lane);
+            const long long t0 = clock64();
+            while (true) {
+                a = __ldcg(hp);
+                b = __ldcg(hp + 1);
+                ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
+                if (ok) break;
+                if (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+                    if (lane == 0) give_up(status, 56, dead);
+                    break;
+                }
+                __nanosleep(128);
             }
-            __nanosleep(256);
         }
+        const float4 v = make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x),
+                                     __uint_as_float(b.z));
         const float mx = digits128(v, lane, sc);
         __syncwarp();
 #pragma unroll
@@ -795,40 +792,47 @@ __device__ __forceinline__ BlobOff blob_off(int H, int I)
     return o;
 }
 
-// Top-k of lt[0..E) in shared memory, as select.cuh's topk_warp_keys (keys, ties to the
-// lower index): lane s < k returns selection s.
-template <int MAXPL>
+// Top-k of lt[0..E) in shared memory (E <= 1024; descending, ties to the lower index):
+// lane s < k returns selection s.  Lane j owns elements j + 32 i; it keeps the best key of
+// its elements not yet taken (a bitmask of taken ones) and rescans them only when its best
+// is the one taken.  Absent and taken elements have key 0, which no value maps to.
+__device__ __forceinline__ void topk_best(const float* lt, int E, int npl, int lane, uint32_t taken,
+                                          uint32_t& bk, int& bi)
+{
+    bk = 0u;
+    bi = 0;
+#pragma unroll 8
+    for (int i = 0; i < npl; i++) {
+        const int e = lane + 32 * i;
+        const uint32_t kk = (e < E && !((taken >> i) & 1u)) ? order_key(lt[e]) : 0u;
+        if (kk > bk) {
+            bk = kk;
+            bi = i;
+        }
+    }
+}
+
 __device__ __forceinline__ void topk_smem(const float* lt, int E, int k, int lane, int& e_out,
                                           uint32_t& key_out)
 {
-    uint32_t key[MAXPL];
-#pragma unroll
-    for (int i = 0; i < MAXPL; i++) {
-        const int e = lane + 32 * i;
-        key[i] = (e < E) ? order_key(lt[e]) : 0u;
-    }
+    const int npl = (E + 31) >> 5;
+    uint32_t taken = 0u, bk;
+    int bi;
+    topk_best(lt, E, npl, lane, taken, bk, bi);
     uint32_t mine = 0u;
     int mine_e = 0;
+#pragma unroll 1
     for (int s = 0; s < k; s++) {
-        uint32_t bk = key[0];
-        int bi = 0;
-#pragma unroll
-        for (int i = 1; i < MAXPL; i++)
-            if (key[i] > bk) {
-                bk = key[i];
-                bi = i;
-            }
         const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
         const uint32_t cand = (bk == m) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
         const uint32_t e = __reduce_min_sync(0xffffffffu, cand);
-        if ((int)(e & 31u) == lane) {
-#pragma unroll
-            for (int i = 0; i < MAXPL; i++)
-                if (i == (int)(e >> 5)) key[i] = 0u;
-        }
         if (lane == s) {
             mine = m;
             mine_e = (int)e;
+        }
+        if ((int)(e & 31u) == lane) {
+            taken |= 1u << (e >> 5);
+            topk_best(lt, E, npl, lane, taken, bk, bi);
         }
     }
     e_out = mine_e;
@@ -847,74 +851,125 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane)
     return x - v;
 }
 
+// Top-k from keys held in registers (E <= 256: lane j holds elements j + 32 i, i < 8) by
+// threshold and rank: the k-th largest of the 32 lane maxima is at most the k-th largest
+// key, so every key of the top k is at or above it.  Those candidates (C of them, about
+// k) go to shared memory and each one's rank among them is counted: larger keys, and equal
+// keys of a lower index, come first; a candidate's rank among the candidates is its rank
+// among all keys.  Key 0 marks an absent element.  When C is above kTopkCand (many equal
+// keys), the sequential selection over lt decides instead.
+constexpr int kTopkCand = 128;
+
+__device__ __forceinline__ void topk_regs(const uint32_t (&key)[8], const float* lt, int E, int k, int lane,
+                                          uint2* cand, uint2* res, int& e_out, uint32_t& key_out)
+{
+    uint32_t lm = key[0];
+#pragma unroll
+    for (int i = 1; i < 8; i++) lm = max(lm, key[i]);
+    int r = 0;
+#pragma unroll
+    for (int j = 0; j < 32; j++) {
+        const uint32_t o = __shfl_sync(0xffffffffu, lm, j);
+        r += (o > lm || (o == lm && j < lane)) ? 1 : 0;
+    }
+    const uint32_t tau = __shfl_sync(0xffffffffu, lm, __ffs(__ballot_sync(0xffffffffu, r == k - 1)) - 1);
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) cnt += (key[i] != 0u && key[i] >= tau) ? 1 : 0;
+    const int pre = warp_excl_scan(cnt, lane);
+    const int C = __shfl_sync(0xffffffffu, pre + cnt, 31);
+    if (C > kTopkCand) {
+        topk_smem(lt, E, k, lane, e_out, key_out);
+        return;
+    }
+    int pos = pre;
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        if (key[i] != 0u && key[i] >= tau) cand[pos++] = make_uint2(key[i], (uint32_t)(lane + 32 * i));
+    __syncwarp();
+#pragma unroll 1
+    for (int ci = lane; ci < C; ci += 32) {
+        const uint2 me = cand[ci];
+        int rank = 0;
+#pragma unroll 4
+        for (int j = 0; j < C; j++) {
+            const uint2 o = cand[j];
+            rank += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        if (rank < k) res[rank] = me;
+    }
+    __syncwarp();
+    const uint2 mine = lane < k ? res[lane] : make_uint2(0u, 0u);
+    e_out = (int)mine.y;
+    key_out = mine.x;
+    __syncwarp();
+}
+
 // Union of sel[t * k + s] (T * k <= 128 assignments, each token's experts distinct and in
-// [0, E)): writes the routed segments of the table (after n_shared leading segments) and,
-// when `out` is set, union_ids / n_union / offsets / assign.  bits: T * 32 words scratch.
+// [0, E)) in ascending expert order: writes the routed segments of the table (after
+// n_shared leading segments) and, when `out` is set, union_ids / n_union / offsets / assign.
+// Scratch `bits`: per token 32 words of expert bits, then per expert word its union prefix,
+// union bits and the number of assignments in lower words.
 __device__ __forceinline__ void build_union(const int* sel, const float* selw, int T, int k, int E, int ns,
                             uint32_t* bits, Table tb, bool out, const FusedParams& p, int lane)
 {
     const int nw = (E + 31) / 32;
     const int n = T * k;
+    uint32_t* wp = bits + kFusedMaxT * 32;
+#pragma unroll 1
     for (int i = lane; i < kFusedMaxT * 32; i += 32) bits[i] = 0u;
     __syncwarp();
+#pragma unroll 1
     for (int a = lane; a < n; a += 32) {
         const int e = sel[a];
         atomicOr(&bits[(a / k) * 32 + (e >> 5)], 1u << (e & 31));
     }
     __syncwarp();
-    // per word w (lane w < nw): union word, and per token the prefix popcounts
     uint32_t uw = 0u;
-    int pre_t[kFusedMaxT];
-    int cnt_below = 0;   // assignments with a smaller expert word, all tokens
-#pragma unroll
-    for (int t = 0; t < kFusedMaxT; t++) {
-        const uint32_t bw = (t < T && lane < nw) ? bits[t * 32 + lane] : 0u;
+    int cw = 0;
+#pragma unroll 1
+    for (int t = 0; t < T; t++) {
+        const uint32_t bw = lane < nw ? bits[t * 32 + lane] : 0u;
         uw |= bw;
-        pre_t[t] = warp_excl_scan(__popc(bw), lane);
-        cnt_below += pre_t[t];
+        cw += __popc(bw);
     }
     const int upre = warp_excl_scan(__popc(uw), lane);
     const int nu = __shfl_sync(0xffffffffu, upre + __popc(uw), 31);
-    for (int a0 = 0; a0 < n; a0 += 32) {
-        const int a = a0 + lane;
-        const bool valid = a < n;
-        const int e = valid ? sel[a] : 0;
-        const int t = valid ? a / k : 0;
-        const int w = e >> 5;
+    wp[lane] = (uint32_t)upre;
+    wp[32 + lane] = uw;
+    wp[64 + lane] = (uint32_t)warp_excl_scan(cw, lane);
+    __syncwarp();
+#pragma unroll 1
+    for (int a = lane; a < n; a += 32) {
+        const int e = sel[a], t = a / k, w = e >> 5;
         const uint32_t below = (1u << (e & 31)) - 1u;
-        const int up_w = __shfl_sync(0xffffffffu, upre, w);
-        const uint32_t uw_w = __shfl_sync(0xffffffffu, uw, w);
-        int off = __shfl_sync(0xffffffffu, cnt_below, w);
-        int before_t = 0, count = 0;
-#pragma unroll
-        for (int tt = 0; tt < kFusedMaxT; tt++) {
-            if (tt < T) {
-                const uint32_t bw = bits[tt * 32 + w];
-                off += __popc(bw & below);
-                const int hit = (bw >> (e & 31)) & 1;
-                count += hit;
-                if (tt < t) before_t += hit;
+        // rank of the assignment: those of lower experts, then this expert's earlier tokens
+        int off = (int)wp[64 + w], before_t = 0, count = 0;
+#pragma unroll 1
+        for (int tt = 0; tt < T; tt++) {
+            const uint32_t bw = bits[tt * 32 + w];
+            const int hit = (bw >> (e & 31)) & 1;
+            off += __popc(bw & below);
+            count += hit;
+            before_t += tt < t ? hit : 0;
+        }
+        const int u = (int)wp[w] + __popc(wp[32 + w] & below);
+        const int seg = ns + u;
+        if (before_t == 0) {
+            tb.e[seg] = e;
+            tb.cnt[seg] = count;
+            tb.base[seg] = off;
+            if (out) {
+                p.union_ids[u] = e;
+                p.offsets[u] = off;
             }
         }
-        if (valid) {
-            const int u = up_w + __popc(uw_w & below);
-            const int rank = off + before_t;
-            const int seg = ns + u;
-            if (before_t == 0) {
-                tb.e[seg] = e;
-                tb.cnt[seg] = count;
-                tb.base[seg] = off;
-                if (out) {
-                    p.union_ids[u] = e;
-                    p.offsets[u] = off;
-                }
-            }
-            tb.tok[seg * kFusedMaxT + before_t] = t;
-            tb.wt[seg * kFusedMaxT + before_t] = selw[a];
-            if (out) p.assign[rank] = a;
-        }
+        tb.tok[seg * kFusedMaxT + before_t] = t;
+        tb.wt[seg * kFusedMaxT + before_t] = selw[a];
+        if (out) p.assign[off + before_t] = a;
     }
     if (out) {
+#pragma unroll 1
         for (int q = nu + lane; q <= E; q += 32) {
             if (q < E) p.union_ids[q] = -1;
             p.offsets[q] = n;
@@ -1004,6 +1059,7 @@ __device__ __forceinline__ void issue_gu(const FusedParams& p, const Ctx& c, Str
     const uint32_t scb = 8u * ntl * ((uint32_t)H / 32u);
     uint64_t* bar;
     uint8_t* dst = slot_begin(p, c, st, 8u * cr * rowb + 2u * scb, bar);
+#pragma unroll 1
     for (int q = 0; q < 4; q++) {
         const uint64_t r = (uint64_t)i0 + q * cr;
         bulk_g2s_hint(dst + (size_t)q * p.gu_chunk, blob + c.bo.gq + r * rowb, cr * rowb, bar, st.pol);
@@ -1023,6 +1079,7 @@ __device__ __forceinline__ void issue_down(const FusedParams& p, const Ctx& c, S
     const uint64_t a0 = s0 & ~15ull, a1 = (s1 + 15) & ~15ull;
     uint64_t* bar;
     uint8_t* dst = slot_begin(p, c, st, (uint32_t)c.nrows * rowb + (uint32_t)(a1 - a0), bar);
+#pragma unroll 1
     for (int q = 0; q < 4; q++) {
         const int n = dcs(c, q + 1) - dcs(c, q);
         if (n > 0)
@@ -1060,41 +1117,69 @@ __device__ __forceinline__ void route_compute(const FusedParams& p, const Ctx& c
     int* sel = reinterpret_cast<int*>(lt + T * E);
     float* selw = reinterpret_cast<float*>(sel + T * k);
     uint32_t* bits = reinterpret_cast<uint32_t*>(selw + T * k);
+    // top-k candidates and results (8-byte aligned)
+    uint2* cand = reinterpret_cast<uint2*>((reinterpret_cast<uintptr_t>(bits + (kFusedMaxT + 3) * 32) + 7) & ~uintptr_t(7));
     const bool out = c.b == 0 && !dry;
+    // the launch generation straight from the workspace (read after the dependency wait)
+    const uint32_t ep = __ldcg(p.gen) * 32u + (uint32_t)l + 1u;
+    int e_sel = 0;
+    float wv = 0.0f;
+#pragma unroll 1
     for (int t = 0; t < T; t++) {
-        for (int e0 = 0; e0 < E; e0 += 32 * 2) {
-            double part[2][8];
+        uint32_t key[8];
+#pragma unroll 1
+        for (int e0 = 0; e0 < E; e0 += 32 * 8) {
+            // the partials of eight experts per lane and their biases in one round of loads
+            double v[8];
+            float bv[8];
 #pragma unroll
-            for (int i = 0; i < 2; i++) {
+            for (int i = 0; i < 8; i++) {
                 const int e = e0 + 32 * i + lane;
+                v[i] = 0.0;
+                bv[i] = (ly.bias && e < E) ? __ldg(ly.bias + e) : 0.0f;
+            }
+#pragma unroll 1
+            for (int cc = 0; cc < p.RC; cc++) {
+                // poll until every partial carries this layer's epoch (the dry pass takes
+                // whatever is there)
+                uint4 q[8];
+                const long long t0 = clock64();
+                while (true) {
 #pragma unroll
-                for (int cc = 0; cc < 8; cc++)
-                    part[i][cc] = (e < E && cc < p.RC) ? __ldcg(p.rpart + ((size_t)t * E + e) * p.RC + cc) : 0.0;
+                    for (int i = 0; i < 8; i++) {
+                        const int e = e0 + 32 * i + lane;
+                        q[i] = e < E ? __ldcg(p.rpart + ((size_t)t * E + e) * p.RC + cc) : make_uint4(0u, ep, 0u, ep);
+                    }
+                    bool ok = true;
+#pragma unroll
+                    for (int i = 0; i < 8; i++) ok = ok && q[i].y == ep && q[i].w == ep;
+                    if (dry || __all_sync(0xffffffffu, ok)) break;
+                    if (*c.dead || timed_out(p.status) || clock64() - t0 > kWaitBudgetCycles) {
+                        if (lane == 0) give_up(p.status, 41, c.dead);
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; i++) v[i] += __hiloint2double((int)q[i].z, (int)q[i].x);
             }
 #pragma unroll
-            for (int i = 0; i < 2; i++) {
+            for (int i = 0; i < 8; i++) {
                 const int e = e0 + 32 * i + lane;
+                const float lv = (float)(v[i] + (double)bv[i]);
+                key[i] = e < E ? order_key(lv) : 0u;
                 if (e < E) {
-                    double sum = 0.0;
-#pragma unroll
-                    for (int cc = 0; cc < 8; cc++)
-                        if (cc < p.RC) sum += part[i][cc];
-                    if (ly.bias) sum += (double)__ldg(ly.bias + e);
-                    const float v = (float)sum;
-                    if (!dry && !isfinite(v)) set_flag(p.status, DEV_NONFINITE);
-                    lt[t * E + e] = v;
-                    if (out && p.logits) p.logits[(size_t)t * E + e] = v;
+                    if (!dry && !isfinite(lv)) set_flag(p.status, DEV_NONFINITE);
+                    lt[t * E + e] = lv;
+                    if (out && p.logits) p.logits[(size_t)t * E + e] = lv;
                 }
             }
         }
-    }
-    __syncwarp();
-    for (int t = 0; t < T; t++) {
-        int e_sel;
-        uint32_t key;
-        if (E <= 256) topk_smem<8>(lt + t * E, E, k, lane, e_sel, key);
-        else topk_smem<32>(lt + t * E, E, k, lane, e_sel, key);
-        const float wv = topk_weight_f(key, k, lane);
+        __syncwarp();
+        uint32_t kv;
+        if (E <= 256) topk_regs(key, lt + t * E, E, k, lane, cand, cand + kTopkCand, e_sel, kv);
+        else topk_smem(lt + t * E, E, k, lane, e_sel, kv);
+        wv = topk_weight_f(kv, k, lane);
         if (lane < k) {
             sel[t * k + lane] = e_sel;
             selw[t * k + lane] = wv;
@@ -1104,19 +1189,59 @@ __device__ __forceinline__ void route_compute(const FusedParams& p, const Ctx& c
         }
     }
     __syncwarp();
-    build_union(sel, selw, T, k, E, ns, bits, tb, out && p.union_ids != nullptr, p, lane);
+    if (T == 1) {
+        // one token: the union is its k experts in ascending id order, one row each
+        int r = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; j++) {
+            const int ej = __shfl_sync(0xffffffffu, e_sel, j);
+            r += (j < k && ej < e_sel) ? 1 : 0;
+        }
+        const bool uo = out && p.union_ids != nullptr;
+        if (lane < k) {
+            const int seg = ns + r;
+            tb.e[seg] = e_sel;
+            tb.cnt[seg] = 1;
+            tb.base[seg] = r;
+            tb.tok[seg * kFusedMaxT] = 0;
+            tb.wt[seg * kFusedMaxT] = wv;
+            if (uo) {
+                p.union_ids[r] = e_sel;
+                p.offsets[r] = r;
+                p.assign[r] = lane;
+            }
+        }
+        if (uo) {
+            for (int q = k + lane; q <= E; q += 32) {
+                if (q < E) p.union_ids[q] = -1;
+                p.offsets[q] = k;
+            }
+            if (lane == 0) *p.n_union = k;
+        }
+        if (lane == 0) {
+            tb.hdr[0] = ns + k;
+            tb.hdr[1] = k;
+        }
+    } else {
+        build_union(sel, selw, T, k, E, ns, bits, tb, out && p.union_ids != nullptr, p, lane);
+    }
     __syncwarp();
 }
 
-__device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, int l)
+// warm: first run the routing code once on whatever the buffers hold (into the other
+// layer's table, which is rewritten before use), so that the real pass finds its code in
+// the instruction caches; both passes go through one copy of the code.
+__device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, int l, bool warm)
 {
     const int T = p.T, E = p.E, k = p.k, ns = p.n_shared, lane = c.lane;
     const Table tb = layer_table(c, l);
     uint32_t* lc = layer_cnt(p, l);
     if (p.route) {
-        if (lane == 0) gwait(&lc[0], (uint32_t)c.n_ritems, p.status, 41, c.dead);
-        __syncwarp();
-        route_compute(p, c, l, tb, false);
+#pragma unroll 1
+        for (int pass = warm ? 0 : 1; pass < 2; pass++) {
+            const bool dry = pass == 0;
+            route_compute(p, c, l, dry ? layer_table(c, l + 1) : tb, dry);
+        }
     } else {
         // given routing (forward call): union_ids / n_union / offsets / assign / w
         int nu = __ldcg(p.n_union);
@@ -1124,6 +1249,7 @@ __device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, 
             if (lane == 0) set_flag(p.status, DEV_BAD_INDEX);
             nu = max(0, min(nu, min(E, T * k)));
         }
+#pragma unroll 1
         for (int u = lane; u < nu; u += 32) {
             const int seg = ns + u;
             int e = __ldcg(p.union_ids + u);
@@ -1137,6 +1263,7 @@ __device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, 
             tb.e[seg] = e;
             tb.cnt[seg] = o1 - o0;
             tb.base[seg] = o0;
+#pragma unroll 1
             for (int m = 0; m < o1 - o0; m++) {
                 int a = __ldcg(p.assign + o0 + m);
                 if (a < 0 || a >= T * k) {
@@ -1156,49 +1283,52 @@ __device__ __forceinline__ void route_layer(const FusedParams& p, const Ctx& c, 
     if (lane == 0) mbar_arrive(&c.hd->route_bar);
 }
 
-// The control warp's order of stages (the consumers follow the same order): router items,
-// the shared expert's gate/up stages of this CTA and its down rows, [routing], the routed
-// gate/up stages of this CTA (one round-robin sequence over all segments' stages), the
-// routed down rows in union order.
+// The control warp's order of stages (the consumers and the reducer follow the same
+// order): router items; the shared expert's gate/up stages of this CTA; [routing]; the
+// routed gate/up stages of this CTA (one round-robin sequence over all segments' stages);
+// the down rows of every segment, the shared expert's first.  Before routing it issues
+// only router items and shared stages (at most the ring's depth at the first layer), then
+// routes; every issue goes through one call site per kind of stage.
 __device__ __forceinline__ void control_warp(const FusedParams& p, const Ctx& c)
 {
     Stream st;
     st.it = 0;
     st.pol = policy_evict_first();
     const int ns = p.n_shared;
+#pragma unroll 1
     for (int l = 0; l < p.L; l++) {
         const FusedLayer& ly = p.layer[l];
-        if (c.lane == 0) {
-            if (c.ri1 > c.ri0) issue_router(p, c, st, ly);
-            if (ns) {
-                for (int gi = c.b; gi < p.SPS; gi += c.G) issue_gu(p, c, st, ly.shared, gi);
-                if (c.nrows > 0) issue_down(p, c, st, ly.shared);
+        const Table tb = layer_table(c, l);
+        if (c.lane == 0 && c.ri1 > c.ri0) issue_router(p, c, st, ly);
+        int nseg = ns, gi = c.b, ds = 0;
+        bool routed = false;
+        while (true) {
+            if (gi < nseg * p.SPS) {
+                const int sg = gi / p.SPS;
+                if (c.lane == 0)
+                    issue_gu(p, c, st, sg < ns ? ly.shared : ly.experts + (uint64_t)tb.e[sg] * ly.stride,
+                             gi - sg * p.SPS);
+                gi += c.G;
+            } else if (!routed) {
+                __syncwarp();
+                if (l == 0) pdl_wait();
+                route_layer(p, c, l, l == 0);
+                nseg = tb.hdr[0];
+                routed = true;
+            } else if (c.nrows > 0 && ds < nseg) {
+                if (c.lane == 0)
+                    issue_down(p, c, st, ds < ns ? ly.shared : ly.experts + (uint64_t)tb.e[ds] * ly.stride);
+                ds++;
+            } else {
+                break;
             }
-        }
-        __syncwarp();
-        if (l == 0) {
-            pdl_wait();
-            // warm the routing code path while the router items are still being computed
-            if (p.route && p.L > 0) route_compute(p, c, l, layer_table(c, l + 1), true);
-        }
-        route_layer(p, c, l);
-        if (c.lane == 0) {
-            const Table tb = layer_table(c, l);
-            const int nseg = tb.hdr[0];
-            int gi = c.b;
-            while (gi < ns * p.SPS) gi += c.G;
-            for (; gi < nseg * p.SPS; gi += c.G) {
-                const int s = gi / p.SPS;
-                issue_gu(p, c, st, ly.experts + (uint64_t)tb.e[s] * ly.stride, gi - s * p.SPS);
-            }
-            if (c.nrows > 0)
-                for (int s = ns; s < nseg; s++) issue_down(p, c, st, ly.experts + (uint64_t)tb.e[s] * ly.stride);
         }
         __syncwarp();
     }
     // drain: every issued copy has landed before the CTA may exit (bounded)
     if (c.lane == 0) {
         const uint32_t n_last = st.it < (uint32_t)p.nslot ? st.it : (uint32_t)p.nslot;
+#pragma unroll 1
         for (uint32_t q = 0; q < n_last; q++) {
             const uint32_t last = st.it - 1 - q;
             const uint32_t s = last % (uint32_t)p.nslot;
@@ -1222,6 +1352,22 @@ struct Cons {
     int d_rs, d_kw, gbase_d, gpw_d;   // down
 };
 
+// One token's h row `base` (I values with their epochs) into staging buffer buf & 1 by
+// asynchronous copies (each warp the 128-value pieces it digitizes), as one commit group.
+__device__ __forceinline__ void h_prefetch(const FusedParams& p, const Ctx& c, int base, uint32_t buf)
+{
+    const int I = p.I;
+    const uint2* row = reinterpret_cast<const uint2*>(p.h) + (size_t)base * I;
+    uint2* stg = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_hstage + (size_t)(buf & 1u) * 8u * I);
+#pragma unroll 1
+    for (int pp = c.warp; pp < I / 128; pp += NCW) {
+        const int o = 128 * pp + 4 * c.lane;
+        cp_async16(stg + o, row + o);
+        cp_async16(stg + o + 2, row + o + 2);
+    }
+    cp_async_commit();
+}
+
 __device__ __forceinline__ const uint8_t* cslot_wait(const FusedParams& p, const Ctx& c, Cons& w)
 {
     const uint32_t s = w.it % (uint32_t)p.nslot;
@@ -1236,77 +1382,181 @@ __device__ __forceinline__ void cslot_free(const FusedParams& p, const Ctx& c, C
     w.it++;
 }
 
-// router items of this CTA: partial logits in double over the item's columns
+// Router items of this CTA, partial logits in double.  Every consumer thread takes a share
+// of every item (float4 j of the item's columns goes to thread j % NCT); the warps' sums
+// per (item, token) are then added in warp order by one thread, so each partial logit has
+// one fixed summation order.  With one item per router row (RC = 1) the normalised input is
+// loaded once per token and kept in registers across the items.
+template <bool PAIR>
 __device__ __forceinline__ void router_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
                                                const float* xin)
 {
     const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
-    const int T = p.T, E = p.E, H = p.H, RKc = p.RKc, RC = p.RC, lane = c.lane;
+    const int T = p.T, E = p.E, H = p.H, RKc = p.RKc, RC = p.RC, lane = c.lane, tid = c.tid;
+    const int nit = c.ri1 - c.ri0, n4 = RKc / 4;
+    constexpr int U = 4;   // float4 per thread per item (RKc <= 4 NCT * 4 = 6144 columns)
+    double* part = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_scratch);
     const uint8_t* sb = cslot_wait(p, c, w);
-    int mine = 0;
-    constexpr int U = 4;   // float4 per lane per pass
-    for (int i = c.ri0 + c.warp; i < c.ri1; i += NCW) {
-        const int e = i / RC, cc = i - e * RC;
-        const float4* wr = reinterpret_cast<const float4*>(sb + (size_t)(i - c.ri0) * RKc * 4);
 #pragma unroll 1
-        for (int t = 0; t < T; t++) {
-            const double r = c.hd->rnorm[t];
-            double acc = 0.0;
-            for (int u0 = 0; u0 < RKc / 4; u0 += 32 * U) {
-                float4 xv[U];
+    for (int t = 0; t < T; t++) {
+        const double r = c.hd->rnorm[t];
+        float4 nv[U];
+        int cc_have = -1;
+#pragma unroll 1
+        for (int it = 0; it < nit; it++) {
+            const int i = c.ri0 + it, e = i / RC, cc = i - e * RC;
+            if constexpr (PAIR) {
+              if (cc != cc_have) {
+                // one token: n is in shared memory already
+                const float4* xs = reinterpret_cast<const float4*>(reinterpret_cast<const uint8_t*>(c.hd) + p.off_hstage);
 #pragma unroll
                 for (int j = 0; j < U; j++) {
-                    const int u = u0 + 32 * j + lane;
-                    xv[j] = u < RKc / 4 ? __ldcg(reinterpret_cast<const float4*>(xin + (size_t)t * H + cc * RKc + 4 * u))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const int u = tid + NCT * j;
+                    nv[j] = u < n4 ? xs[cc * (RKc / 4) + u] : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+                cc_have = cc;
+              }
+            } else if (cc != cc_have) {
+                // n = float(x * r * gamma): exactly x for a plain input
 #pragma unroll
                 for (int j = 0; j < U; j++) {
-                    const int u = u0 + 32 * j + lane;
-                    if (u < RKc / 4) {
-                        const float4 wv = wr[u];
-                        float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
-                        if (gamma) gm = __ldg(reinterpret_cast<const float4*>(gamma + cc * RKc + 4 * u));
-                        const float4 x = xv[j];
-                        // n = float(x * r * gamma): exactly x for a plain input
-                        acc = fma((double)(float)((double)x.x * r * (double)gm.x), (double)wv.x, acc);
-                        acc = fma((double)(float)((double)x.y * r * (double)gm.y), (double)wv.y, acc);
-                        acc = fma((double)(float)((double)x.z * r * (double)gm.z), (double)wv.z, acc);
-                        acc = fma((double)(float)((double)x.w * r * (double)gm.w), (double)wv.w, acc);
+                    const int u = tid + NCT * j;
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), gm = make_float4(1.f, 1.f, 1.f, 1.f);
+                    if (u < n4) {
+                        x = __ldcg(reinterpret_cast<const float4*>(xin + (size_t)t * H + cc * RKc) + u);
+                        if (gamma) gm = __ldg(reinterpret_cast<const float4*>(gamma + cc * RKc) + u);
                     }
+                    nv[j].x = (float)((double)x.x * r * (double)gm.x);
+                    nv[j].y = (float)((double)x.y * r * (double)gm.y);
+                    nv[j].z = (float)((double)x.z * r * (double)gm.z);
+                    nv[j].w = (float)((double)x.w * r * (double)gm.w);
+                }
+                cc_have = cc;
+            }
+            const float4* wr = reinterpret_cast<const float4*>(sb + (size_t)it * RKc * 4);
+            double acc = 0.0;
+#pragma unroll
+            for (int j = 0; j < U; j++) {
+                const int u = tid + NCT * j;
+                if (u < n4) {
+                    const float4 wv = wr[u];
+                    acc = fma((double)nv[j].x, (double)wv.x, acc);
+                    acc = fma((double)nv[j].y, (double)wv.y, acc);
+                    acc = fma((double)nv[j].z, (double)wv.z, acc);
+                    acc = fma((double)nv[j].w, (double)wv.w, acc);
                 }
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) p.rpart[((size_t)t * E + e) * RC + cc] = acc;
+            if (lane == 0) part[(it * T + t) * NCW + c.warp] = acc;
         }
-        mine++;
     }
     cslot_free(p, c, w);
-    if (lane == 0 && mine > 0) red_release_add(&layer_cnt(p, l)[0], (uint32_t)mine);
+    named_bar(5, NCT);
+    // each partial as two 8-byte (half, epoch) words: a reader polls the values themselves
+    const uint32_t ep = h_epoch(c, l);
+    for (int q = tid; q < nit * T; q += NCT) {
+        const int it = q / T, t = q - it * T, i = c.ri0 + it, e = i / RC, cc = i - e * RC;
+        double sum = 0.0;
+#pragma unroll 1
+        for (int ww = 0; ww < NCW; ww++) sum += part[q * NCW + ww];
+        p.rpart[((size_t)t * E + e) * RC + cc] =
+            make_uint4((uint32_t)__double2loint(sum), ep, (uint32_t)__double2hiint(sum), ep);
+    }
+    named_bar(5, NCT);
+}
+
+// One token (pair mode): the layer input once per layer into shared memory as the
+// normalised n = float(x * r * gamma) (exactly x for a plain input), with the RMSNorm
+// factor r and the activation scale 126 / max|n| in the head.  Thread tid holds float4
+// u = tid + NCT j of the row; every thread sums the warps' parts in the same order.
+__device__ __forceinline__ void load_x_pair(const FusedParams& p, const Ctx& c, int l, const float* xin)
+{
+    const int n4 = p.H / 4, tid = c.tid, lane = c.lane, warp = c.warp;
+    const float4* gamma = p.norm ? reinterpret_cast<const float4*>(p.layer[l].gamma) : nullptr;
+    Head& hd = *c.hd;
+    float4* xs = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_hstage);
+    constexpr int U = 4;   // H <= 16 NCT
+    float4 v[U];
+#pragma unroll
+    for (int j = 0; j < U; j++) {
+        const int u = tid + NCT * j;
+        v[j] = u < n4 ? __ldcg(reinterpret_cast<const float4*>(xin) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    double r = 1.0;
+    if (p.norm) {
+        double sq = 0.0;
+#pragma unroll
+        for (int j = 0; j < U; j++) {
+            sq = fma((double)v[j].x, (double)v[j].x, sq);
+            sq = fma((double)v[j].y, (double)v[j].y, sq);
+            sq = fma((double)v[j].z, (double)v[j].z, sq);
+            sq = fma((double)v[j].w, (double)v[j].w, sq);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) hd.rsq[warp][0] = sq;
+        named_bar(5, NCT);
+        double s2 = 0.0;
+#pragma unroll 1
+        for (int ww = 0; ww < NCW; ww++) s2 += hd.rsq[ww][0];
+        r = 1.0 / sqrt(s2 / (double)p.H + p.eps);
+    }
+    float mx = 0.0f;
+#pragma unroll
+    for (int j = 0; j < U; j++) {
+        const int u = tid + NCT * j;
+        if (u < n4) {
+            const float4 gm = gamma ? __ldg(gamma + u) : make_float4(1.f, 1.f, 1.f, 1.f);
+            float4 n;
+            n.x = (float)((double)v[j].x * r * (double)gm.x);
+            n.y = (float)((double)v[j].y * r * (double)gm.y);
+            n.z = (float)((double)v[j].z * r * (double)gm.z);
+            n.w = (float)((double)v[j].w * r * (double)gm.w);
+            xs[u] = n;
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(n.x), fabsf(n.y)), fmaxf(fabsf(n.z), fabsf(n.w))));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) hd.amax[warp][0] = mx;
+    named_bar(5, NCT);
+    if (tid == 0) {
+        float m2 = 0.0f;
+        for (int ww = 0; ww < NCW; ww++) m2 = fmaxf(m2, hd.amax[ww][0]);
+        hd.rnorm[0] = r;
+        hd.xinv[0] = m2 > 0.0f ? 126.0f / m2 : 0.0f;
+        hd.xfac[0] = m2 * (1.0f / 126.0f);
+    }
+    named_bar(5, NCT);
 }
 
 // RMSNorm factors (stacks; 1 otherwise) and the per-token activation scale of the layer
 // input; every CTA sums in the same order, so all CTAs agree bit for bit
 __device__ __forceinline__ void input_scales(const FusedParams& p, const Ctx& c, int l, const float* xin)
 {
-    const int T = p.T, H = p.H, tid = c.tid, lane = c.lane, warp = c.warp;
-    const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
+    const int T = p.T, n4 = p.H / 4, tid = c.tid, lane = c.lane, warp = c.warp;
+    const float4* gamma = p.norm ? reinterpret_cast<const float4*>(p.layer[l].gamma) : nullptr;
     Head& hd = *c.hd;
-    constexpr int U = 16;   // values per thread per pass (H <= 6144 in one pass)
+    constexpr int U = 4;   // float4 per thread per pass (H <= 6144 in one pass)
     if (p.norm) {
 #pragma unroll 1
         for (int t = 0; t < T; t++) {
+            const float4* xr = reinterpret_cast<const float4*>(xin + (size_t)t * p.H);
             double sq = 0.0;
-            for (int c0 = 0; c0 < H; c0 += NCT * U) {
-                float xv[U];
+#pragma unroll 1
+            for (int i0 = tid; i0 < n4; i0 += NCT * U) {
+                float4 v[U];
+#pragma unroll
+                for (int j = 0; j < U; j++)
+                    v[j] = i0 + NCT * j < n4 ? __ldcg(xr + i0 + NCT * j) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < U; j++) {
-                    const int cc = c0 + NCT * j + tid;
-                    xv[j] = cc < H ? __ldcg(xin + (size_t)t * H + cc) : 0.0f;
+                    sq = fma((double)v[j].x, (double)v[j].x, sq);
+                    sq = fma((double)v[j].y, (double)v[j].y, sq);
+                    sq = fma((double)v[j].z, (double)v[j].z, sq);
+                    sq = fma((double)v[j].w, (double)v[j].w, sq);
                 }
-#pragma unroll
-                for (int j = 0; j < U; j++) sq = fma((double)xv[j], (double)xv[j], sq);
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -1315,27 +1565,32 @@ __device__ __forceinline__ void input_scales(const FusedParams& p, const Ctx& c,
         named_bar(5, NCT);
         if (tid < T) {
             double sq = 0.0;
+#pragma unroll 1
             for (int w = 0; w < NCW; w++) sq += hd.rsq[w][tid];
-            hd.rnorm[tid] = 1.0 / sqrt(sq / (double)H + p.eps);
+            hd.rnorm[tid] = 1.0 / sqrt(sq / (double)p.H + p.eps);
         }
         named_bar(5, NCT);
     }
 #pragma unroll 1
     for (int t = 0; t < T; t++) {
+        const float4* xr = reinterpret_cast<const float4*>(xin + (size_t)t * p.H);
         float mx = 0.0f;
         const double r = p.norm ? hd.rnorm[t] : 1.0;
-        for (int c0 = 0; c0 < H; c0 += NCT * U) {
-            float xv[U];
+#pragma unroll 1
+        for (int i0 = tid; i0 < n4; i0 += NCT * U) {
+            float4 v[U];
+#pragma unroll
+            for (int j = 0; j < U; j++)
+                v[j] = i0 + NCT * j < n4 ? __ldcg(xr + i0 + NCT * j) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < U; j++) {
-                const int cc = c0 + NCT * j + tid;
-                xv[j] = cc < H ? __ldcg(xin + (size_t)t * H + cc) : 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < U; j++) {
-                const int cc = c0 + NCT * j + tid;
-                const double gm = (gamma && cc < H) ? (double)__ldg(gamma + cc) : 1.0;
-                mx = fmaxf(mx, fabsf((float)((double)xv[j] * r * gm)));
+                // n = float(x * r * gamma): exactly x for a plain input
+                float4 gm = make_float4(1.f, 1.f, 1.f, 1.f);
+                if (gamma && i0 + NCT * j < n4) gm = __ldg(gamma + i0 + NCT * j);
+                mx = fmaxf(mx, fabsf((float)((double)v[j].x * r * (double)gm.x)));
+                mx = fmaxf(mx, fabsf((float)((double)v[j].y * r * (double)gm.y)));
+                mx = fmaxf(mx, fabsf((float)((double)v[j].z * r * (double)gm.z)));
+                mx = fmaxf(mx, fabsf((float)((double)v[j].w * r * (double)gm.w)));
             }
         }
 #pragma unroll
@@ -1345,6 +1600,7 @@ __device__ __forceinline__ void input_scales(const FusedParams& p, const Ctx& c,
     named_bar(5, NCT);
     if (tid < T) {
         float mx = 0.0f;
+#pragma unroll 1
         for (int w = 0; w < NCW; w++) mx = fmaxf(mx, hd.amax[w][tid]);
         hd.xinv[tid] = mx > 0.0f ? 126.0f / mx : 0.0f;
         hd.xfac[tid] = mx * (1.0f / 126.0f);
@@ -1361,7 +1617,8 @@ __device__ __forceinline__ void build_x_operand(const FusedParams& p, const Ctx&
     const Head& hd = *c.hd;
     const float* gamma = p.norm ? p.layer[l].gamma : nullptr;
     if constexpr (PAIR) {
-        build_x_pairs<GPWG, NTM>(xin, hd.xinv[0], hd.rnorm[0], gamma, w.gbase_g, w.gpw_g, w.sc, c.lane, Bx);
+        build_x_pairs<GPWG, NTM>(reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(c.hd) + p.off_hstage),
+                                 hd.xinv[0], w.gbase_g, w.gpw_g, w.sc, c.lane, Bx);
     } else {
 #pragma unroll
         for (int q = 0; q < NTM; q++) {
@@ -1389,11 +1646,13 @@ __device__ __forceinline__ void gu_consume(const FusedParams& p, const Ctx& c, C
     const int ntl = min(p.NTSg, (I - i0) / 8);
     const int cr = 2 * ntl;    // rows per chunk
     uint32_t qmask = 0;
+#pragma unroll 1
     for (int m = 0; m < sg.c; m++) qmask |= 1u << (sg.tok[m] >> 1);
     red_wait_free(*c.hd, w.cs, p.status, c.dead, lane);
     float* rb = c.red + (size_t)(w.cs % kRedBufs) * p.red_floats;
     const int g = lane >> 2, t = lane & 3;
     const uint32_t rowb = (uint32_t)H / 2, srow = (uint32_t)H / 64;
+#pragma unroll 1
     for (int tl = w.g_rs; tl < ntl; tl += p.RSg) {
         // lane row g: chunk g & 3, row 2 tl + (g >> 2) of the chunk
         const int lr = 2 * tl + (g >> 2);
@@ -1421,7 +1680,7 @@ __device__ __forceinline__ void gu_consume(const FusedParams& p, const Ctx& c, C
 // the down stage of segment s (this CTA's output rows), combined into yacc
 template <int NTM, int GPWD, bool PAIR>
 __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
-                                             const Seg& sg, uint32_t (&Bh)[GPWD][NTM][4],
+                                             const Seg& sg, int next_base, uint32_t (&Bh)[GPWD][NTM][4],
                                              float (&fh)[GPWD][NTM])
 {
     const int T = p.T, I = p.I, lane = c.lane;
@@ -1429,11 +1688,22 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
     const uint32_t ep = h_epoch(c, l);
     const uint2* hb = reinterpret_cast<const uint2*>(p.h);
     if constexpr (PAIR) {
-        // the segment's h digits once per CTA (double-buffered), then each warp's operand
+        // the segment's h digits once per CTA (double-buffered), then each warp's operand.
+        // h arrives by asynchronous copies issued one segment ahead (staging buffer
+        // ds & 1); the next segment's copies are issued before this one's are awaited
         uint8_t* hd0 = reinterpret_cast<uint8_t*>(c.hd) + p.off_hdig + (size_t)(w.ds & 1) * p.hdig_bytes;
         uint32_t* dig = reinterpret_cast<uint32_t*>(hd0);
         float* facs = reinterpret_cast<float*>(hd0 + 3 * I);
-        digitize_h_row(hb + (size_t)sg.base * I, ep, I, c.warp, lane, w.sc, dig, facs, p.status, c.dead);
+        if (next_base >= 0) {
+            h_prefetch(p, c, next_base, w.ds + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();
+        const uint2* stg = reinterpret_cast<const uint2*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_hstage +
+                                                          (size_t)(w.ds & 1) * 8u * I);
+        digitize_h_row(stg, hb + (size_t)sg.base * I, ep, I, c.warp, lane, w.sc, dig, facs, p.status, c.dead);
         named_bar(6, NCT);
         gather_h_pairs<GPWD, NTM>(dig, facs, I, w.gbase_d, lane, Bh, fh);
         w.ds++;
@@ -1457,6 +1727,7 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
     const uint32_t rowb = (uint32_t)I / 2, srow = (uint32_t)I / 64;
     const __half* scb = reinterpret_cast<const __half*>(sb + p.d_sc_off + delta);
     const int ntdm = p.ntdm;
+#pragma unroll 1
     for (int tl = w.d_rs; tl < c.ntd; tl += p.RSd) {
         // MMA row m: chunk m & 3, row 4 tl + (m >> 2) of the chunk (rows g and g + 8)
         const int q = g & 3, la = 4 * tl + (g >> 2), lb = la + 2;
@@ -1493,6 +1764,7 @@ __device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, ui
     const int cr = 2 * ntl;
     uint2* hb = reinterpret_cast<uint2*>(p.h);
     const int ntask = ntl * 8 * sg.c, part = lane & 3;
+#pragma unroll 1
     for (int t0 = 0; t0 < ntask; t0 += 8) {
         const int task = t0 + (lane >> 2);
         const bool valid = task < ntask;
@@ -1501,6 +1773,7 @@ __device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, ui
         const int tok = sg.tok[m];
         float gsum = 0.0f, usum = 0.0f;
         if (valid)
+#pragma unroll 1
             for (int kw = part; kw < p.KWg; kw += 4) {
                 const float* q = rb + (size_t)(kw * p.NTSg + tl) * 16 * T;
                 gsum += q[r * T + tok];
@@ -1524,6 +1797,7 @@ __device__ __forceinline__ void reduce_down(const FusedParams& p, const Ctx& c, 
     const int T = p.T, lane = c.lane, cn = sg.c, ntdm = p.ntdm;
     const float* rb = c.red + (size_t)(cs % kRedBufs) * p.red_floats;
     const int ntask = c.ntd * 16 * cn, part = lane & 3;
+#pragma unroll 1
     for (int t0 = 0; t0 < ntask; t0 += 8) {
         const int task = t0 + (lane >> 2);
         const int m = task % cn, rr = task / cn;
@@ -1532,6 +1806,7 @@ __device__ __forceinline__ void reduce_down(const FusedParams& p, const Ctx& c, 
         const bool valid = task < ntask && lrow < dcs(c, q + 1) - dcs(c, q);
         float sum = 0.0f;
         if (valid)
+#pragma unroll 1
             for (int kw = part; kw < p.KWd; kw += 4) sum += rb[((size_t)(kw * ntdm + tl) * 16 + mm) * T + m];
         sum += __shfl_xor_sync(0xffffffffu, sum, 1);
         sum += __shfl_xor_sync(0xffffffffu, sum, 2);
@@ -1542,7 +1817,8 @@ __device__ __forceinline__ void reduce_down(const FusedParams& p, const Ctx& c, 
     }
 }
 
-// The reducer follows the consumers' sequence of reduction stages.
+// The reducer follows the consumers' sequence of reduction stages: the shared gate/up
+// stages of the CTA, [routing], the routed ones, then the down stages of every segment.
 __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c, uint32_t gen)
 {
     const int T = p.T, k = p.k, ns = p.n_shared, lane = c.lane;
@@ -1552,45 +1828,41 @@ __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c,
     sh.tok = c.hd->sh_tok;
     sh.wt = c.hd->sh_wt;
     uint32_t cs = 0;
-    auto take = [&]() {
-        mwait(&c.hd->red_full[cs % kRedBufs], (cs / kRedBufs) & 1u, p.status, 59, c.dead);
-    };
-    auto give = [&]() {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.hd->red_empty[cs % kRedBufs]);
-        cs++;
-    };
+#pragma unroll 1
     for (int l = 0; l < p.L; l++) {
         const uint32_t ep = gen * 32u + (uint32_t)l + 1u;
-        int gi = c.b;
-        if (ns) {
-            for (; gi < p.SPS; gi += c.G) {
-                take();
-                reduce_gu(p, c, cs, sh, gi, ep);
-                give();
+        Table tb;
+        int nseg = ns, gi = c.b, ds = 0;
+        bool routed = false;
+        while (true) {
+            int kind = 0, seg = 0;
+            if (gi < nseg * p.SPS) {
+                kind = 1;
+                seg = gi / p.SPS;
+            } else if (!routed) {
+                mwait(&c.hd->route_bar, (uint32_t)l & 1u, p.status, 60, c.dead);
+                tb = layer_table(c, l);
+                nseg = tb.hdr[0];
+                routed = true;
+                continue;
+            } else if (c.nrows > 0 && ds < nseg) {
+                kind = 2;
+                seg = ds++;
+            } else {
+                break;
             }
-            if (c.nrows > 0) {
-                take();
-                reduce_down(p, c, cs, sh);
-                give();
+            mwait(&c.hd->red_full[cs % kRedBufs], (cs / kRedBufs) & 1u, p.status, 59, c.dead);
+            const Seg sg = seg < ns ? sh : seg_of(tb, seg);
+            if (kind == 1) {
+                reduce_gu(p, c, cs, sg, gi - seg * p.SPS, ep);
+                gi += c.G;
+            } else {
+                reduce_down(p, c, cs, sg);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c.hd->red_empty[cs % kRedBufs]);
+            cs++;
         }
-        mwait(&c.hd->route_bar, (uint32_t)l & 1u, p.status, 60, c.dead);
-        const Table tb = layer_table(c, l);
-        const int nseg = tb.hdr[0];
-        while (gi < ns * p.SPS) gi += c.G;
-        for (; gi < nseg * p.SPS; gi += c.G) {
-            const int sg = gi / p.SPS;
-            take();
-            reduce_gu(p, c, cs, seg_of(tb, sg), gi - sg * p.SPS, ep);
-            give();
-        }
-        if (c.nrows > 0)
-            for (int sg = ns; sg < nseg; sg++) {
-                take();
-                reduce_down(p, c, cs, seg_of(tb, sg));
-                give();
-            }
         // the layer's output rows are summed: the consumers write them, then yacc is clear
         named_bar(7, NCT + 32);
         named_bar(8, NCT + 32);
@@ -1630,6 +1902,7 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
     sh.tok = c.hd->sh_tok;
     sh.wt = c.hd->sh_wt;
 
+#pragma unroll 1
     for (int l = 0; l < p.L; l++) {
         uint32_t* lc = layer_cnt(p, l);
         const float* xin = l == 0 ? p.x : p.xbuf + (size_t)((l - 1) & 1) * T * H;
@@ -1641,14 +1914,24 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
         }
         // the router needs only the RMSNorm factors (1 for a plain input), so for a plain
         // input it runs first and the routing is decided while the scales are formed
-        if (!p.norm && c.ri1 > c.ri0) router_consume(p, c, w, l, xin);
-        input_scales(p, c, l, xin);
-        if (p.norm && c.ri1 > c.ri0) router_consume(p, c, w, l, xin);
+        if constexpr (PAIR) {
+            load_x_pair(p, c, l, xin);
+            if (c.ri1 > c.ri0) router_consume<true>(p, c, w, l, xin);
+        } else {
+#pragma unroll 1
+            for (int step = 0; step < 2; step++) {
+                if ((step == 0) != (p.norm != 0)) {
+                    if (c.ri1 > c.ri0) router_consume<false>(p, c, w, l, xin);
+                } else {
+                    input_scales(p, c, l, xin);
+                }
+            }
+        }
         // stages in the control warp's order; one code path per kind of step
-        //   phase 0: x operand, 1: shared gate/up, 2: shared down, 3: x operand again,
-        //   4: routing, 5: routed gate/up, 6: routed down
+        //   phase 0: x operand, 1: shared gate/up, 4: routing, 5: routed gate/up,
+        //   6: down rows of every segment (the shared expert's first)
         Table tb;
-        int nseg = 0, phase = 0, gi = c.b, sd = ns;
+        int nseg = 0, phase = 0, gi = c.b, sd = 0;
         while (true) {
             int kind = -1, seg = 0, stage = 0;   // 0: x operand, 1: gate/up, 2: down
             if (phase == 0) {
@@ -1661,21 +1944,9 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                     stage = gi;
                     gi += c.G;
                 } else {
-                    phase = 2;
+                    phase = 4;
                     continue;
                 }
-            } else if (phase == 2) {
-                phase = 4;
-                if (ns && c.nrows > 0) {
-                    kind = 2;
-                    seg = 0;
-                    phase = 3;
-                } else {
-                    continue;
-                }
-            } else if (phase == 3) {
-                kind = 0;
-                phase = 4;
             } else if (phase == 4) {
                 mwait(&c.hd->route_bar, (uint32_t)l & 1u, p.status, 55, c.dead);
                 tb = layer_table(c, l);
@@ -1691,6 +1962,10 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                     gi += c.G;
                 } else {
                     phase = 6;
+                    // the first down segment's h on its way into shared memory
+                    if constexpr (PAIR)
+                        if (c.nrows > 0 && nseg > 0)
+                            h_prefetch(p, c, ns ? sh.base : seg_of(tb, 0).base, w.ds);
                     continue;
                 }
             } else {
@@ -1707,17 +1982,22 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                 const Seg sg = seg < ns ? sh : seg_of(tb, seg);
                 if (kind == 1) {
                     gu_consume<NTM, GPWG, PAIR>(p, c, w, l, sg, stage, Bx, fdummy);
-                } else if constexpr (GPWG == GPWD) {
-                    // the h operand takes the x operand's registers (x is rebuilt after the
-                    // shared expert's down stage and not needed after the routed ones)
-                    down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bx, fdummy);
                 } else {
-                    down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bh, fh);
+                    // the base row of the next down segment's h (prefetched), or -1
+                    const int nb = sd < nseg ? (sd < ns ? sh.base : seg_of(tb, sd).base) : -1;
+                    if constexpr (GPWG == GPWD) {
+                        // the h operand takes the x operand's registers (the down stages
+                        // follow every gate/up stage of the layer)
+                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, nb, Bx, fdummy);
+                    } else {
+                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, nb, Bh, fh);
+                    }
                 }
             }
         }
         // ---- this CTA's rows of the layer output (once the reducer has summed them all)
         named_bar(7, NCT + 32);
+#pragma unroll 1
         for (int i = c.tid; i < c.nrows * T; i += NCT) {
             const int rr = i / T, t = i - rr * T;
             const size_t o = (size_t)t * H + c.r0 + rr;
@@ -1762,16 +2042,19 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
 
     pdl_launch_dependents();
     if (c.tid == 0) {
+#pragma unroll 1
         for (int s = 0; s < p.nslot; s++) {
             mbar_init(&c.hd->full[s], 1);
             mbar_init(&c.hd->empty[s], NCW);
         }
         mbar_init(&c.hd->route_bar, 1);
         c.hd->dead = 0;
+#pragma unroll 1
         for (int b2 = 0; b2 < kRedBufs; b2++) {
             mbar_init(&c.hd->red_full[b2], NCW);
             mbar_init(&c.hd->red_empty[b2], 1);
         }
+#pragma unroll 1
         for (int m = 0; m < kFusedMaxT; m++) {
             c.hd->sh_tok[m] = m;
             c.hd->sh_wt[m] = 1.0f;
@@ -1779,6 +2062,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
         }
         fence_barrier_init();
     }
+#pragma unroll 1
     for (int i = c.tid; i < p.rows_max * p.T; i += NTHR) c.yacc[i] = 0.0f;
     __syncthreads();
 
@@ -1800,6 +2084,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
         const uint32_t prev = atomicAdd(&p.cnt[0], 1u);
         if (prev == (uint32_t)c.G - 1u) {
             __threadfence();
+#pragma unroll 1
             for (int i = 1; i < 1 + p.L * kCntPerLayer; i++) p.cnt[i] = 0u;
             *p.gen = c.hd->gen + 1u;
             __threadfence();
@@ -1901,7 +2186,7 @@ bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
     // one token: both matrices in group pairs when each splits into warp shares of exactly 4
     // or 8 aligned groups; the 16-byte row reads need the chunks 64 bytes (mod 128) apart
     p.pair = 0;
-    if (T == 1 && H % 512 == 0 && I % 512 == 0) {
+    if (T == 1 && H % 512 == 0 && I % 512 == 0 && H <= 16 * NCT) {
         const int kg = kw_pair(ngg), kd = kw_pair(ngd);
         if (kg && kd) {
             p.pair = 1;
@@ -1935,13 +2220,22 @@ bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
                        : chunk_stride(4u * p.ntdm * (uint32_t)I / 2u);
     p.d_sc_off = 4u * p.d_chunk;
     const uint32_t d_stage = p.d_sc_off + (uint32_t)(p.rows_max + 16) * (uint32_t)I / 32u + 32u;
-    // router: column chunks so that every CTA gets about one item per consumer warp
+    // router: whole rows per item (RC = 1) when a CTA's rows fit in a weight slot, else
+    // rows in RC column chunks; the consumer threads share every item (at most 16
+    // columns per thread) and the per-warp partial sums of all items fit the scratch
+    uint32_t slot = gu_stage > d_stage ? gu_stage : d_stage;
     p.RC = 1;
-    while (p.RC < 8 && E * p.RC * 2 <= NCW * G && (H / (2 * p.RC)) % 128 == 0) p.RC *= 2;
+    while (true) {
+        const int im = (E * p.RC + G - 1) / G;
+        const bool fits = (uint32_t)im * (uint32_t)(H / p.RC) * 4u <= slot && H / p.RC <= 16 * NCT &&
+                          im * T <= 48;
+        if (fits || (H / (2 * p.RC)) % 128 != 0) break;
+        p.RC *= 2;
+    }
+    if (H / p.RC > 16 * NCT || ((E * p.RC + G - 1) / G) * T > 48) return false;
     p.RKc = H / p.RC;
     const int items_max = (E * p.RC + G - 1) / G;
     const uint32_t r_stage = (uint32_t)items_max * (uint32_t)p.RKc * 4u;
-    uint32_t slot = gu_stage > d_stage ? gu_stage : d_stage;
     if (r_stage > slot) slot = r_stage;
     p.slot_bytes = up128(slot);
     // fixed shared memory: head, two routing tables, partial sums, y rows, scratch
@@ -1957,11 +2251,14 @@ bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
     p.hdig_bytes = p.pair ? (uint32_t)(3 * I + 4 * (I / 64)) : 0u;
     p.off_hdig = off;
     off = up128(off + 2u * p.hdig_bytes);
+    p.off_hstage = off;   // pair mode: two staged h rows (value, epoch)
+    // (the same area holds the layer input row before the down stages)
+    off = up128(off + (p.pair ? (2u * 8u * (uint32_t)I > 4u * (uint32_t)H ? 2u * 8u * (uint32_t)I : 4u * (uint32_t)H) : 0u));
     p.off_scratch = off;
     // consumer digit scratch (96 words per warp), then the control warp's logits,
     // selections, weights and bitmaps
     off = up128(off + NCW * 96u * 4u + (uint32_t)(T * E) * 4u + 2u * (uint32_t)(T * p.k) * 4u +
-                kFusedMaxT * 32u * 4u);
+                (kFusedMaxT + 3) * 32u * 4u + (kTopkCand + 32) * 8u + 8u);
     p.off_ring = off;
     if (off + 2u * p.slot_bytes > smem_limit) return false;
     int nslot = (int)((smem_limit - off) / p.slot_bytes);

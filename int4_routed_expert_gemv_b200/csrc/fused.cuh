@@ -15,7 +15,7 @@ constexpr int kFusedMaxLayers = 16;    // layers per launch (longer stacks: seve
 constexpr int kFusedMaxK = 32;
 constexpr int kFusedMaxSeg = 1 + kFusedMaxT * kFusedMaxK;   // shared expert + union entries
 // counters: word 0 = exit ticket; then per layer kCntPerLayer words:
-//   [0] router items finished, [1] CTAs that wrote their rows of the layer output,
+//   [0] unused, [1] CTAs that wrote their rows of the layer output,
 //   [2 + s] gate/up stages finished of segment s
 constexpr int kCntPerLayer = 2 + kFusedMaxSeg;
 constexpr int kCntWords = 1 + kFusedMaxLayers * kCntPerLayer;
@@ -56,7 +56,7 @@ struct FusedParams {
     uint32_t* status;        // header status word (timeout site at status + 3)
     uint32_t* gen;           // header launch generation (epochs of h)
     uint32_t* cnt;           // kCntWords counters, zero between launches
-    double* rpart;           // [T][E][RC] router partial sums
+    uint4* rpart;            // [T][E][RC] router partial sums: (low word, epoch, high word, epoch)
     uint2* h;                // [T*(k+n_shared)][I] SwiGLU activations as (value, epoch)
     // plan (fused_plan)
     int grid, nslot;
@@ -73,6 +73,7 @@ struct FusedParams {
     uint32_t d_chunk, d_sc_off;          // down stage: chunk stride, scale area
     uint32_t red_floats;                 // one partial-sum buffer
     uint32_t off_hdig, hdig_bytes;       // pair mode: compact h digits, two buffers
+    uint32_t off_hstage;                 // pair mode: two staged h rows
     uint32_t off_red, off_yacc, off_scratch, off_ring;   // dynamic shared memory layout
 };
 
