@@ -47,6 +47,11 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--pool", type=int, default=64, help="distinct token batches rotated over")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--steady", action="store_true",
+                    help="also time back-to-back calls (no flush) rotating over weight copies "
+                         "that together hold at least 3x L2")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations' lines (run by default at N=1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--api", default="layer", choices=["layer", "calls"],
                     help="timed step: one coli_moe_layer call per layer, or the separate "
@@ -236,6 +241,11 @@ def run_ours(args, rank, world, local_rank):
     flush_sink = torch.empty(1, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     slots = 4 if stack else 3          # kernels timed per layer
+    # decode batches (T <= 4) through the layer API run the fused kernel: one launch per
+    # layer, or one launch for the whole stack (coli_moe_stack)
+    fused = args.api == "layer" and T <= 4
+    y_stack = torch.empty(T, H, dtype=torch.float32, device=dev)
+    stack_w = [L_["weights"] for L_ in layers]
 
     def layer_calls(l, x_in, ev, e0):
         """One layer; ev[e0 .. e0+slots] bracket its launches."""
@@ -289,7 +299,10 @@ def run_ours(args, rank, world, local_rank):
         """The step with events only around it (no event nodes between kernels, so
         consecutive launches keep their programmatic dependency)."""
         ev[0].record()
-        if stack:
+        if stack and fused:
+            B.check(B.coli_moe_stack(dims, stack_w, [gamma] * NL, 1e-5, xs[i % R], T, None, y_stack,
+                                     bufs.ws), "coli_moe_stack")
+        elif stack:
             x_work.copy_(xs[i % R])
             for l in range(NL):
                 one_layer(l, x_work)
@@ -399,7 +412,10 @@ def run_ours(args, rank, world, local_rank):
 
         def e2e_step(i):
             xin.copy_(xs_host[i % R], non_blocking=True)
-            if stack:
+            if stack and fused:
+                B.check(B.coli_moe_stack(dims, stack_w, [gamma] * NL, 1e-5, xin, T, None, y_stack, bufs.ws))
+                y_host.copy_(y_stack, non_blocking=True)
+            elif stack:
                 for l in range(NL):
                     B.check(B.coli_rmsnorm(H, T, xin, gamma, 1e-5, n_work))
                     B.check(B.coli_moe_layer(dims, layers[l]["weights"], n_work, T, bufs.idx,
@@ -458,6 +474,15 @@ def run_ours(args, rank, world, local_rank):
         kernels["rmsnorm"] = {"avg_us": round(float(rms_ms.mean()) * 1e3, 3),
                               "share": round(float(rms_ms.sum() / step_ms.sum()), 4)}
     dom = max((n for n in kernels if n != "rmsnorm"), key=lambda n: kernels[n]["share"])
+    if fused:
+        # the timed step is one launch of the fused kernel: its bytes over its duration
+        fgbs = float(step_bytes.sum() / (total_ms * 1e-3) / 1e9)
+        kernels = {"fused_moe_kernel": {"avg_us": round(total_ms / K * 1e3, 3),
+                                        "bytes_per_launch": float(step_bytes.mean()),
+                                        "gb_s": round(fgbs, 1), "frac": round(fgbs / peak, 4),
+                                        "share": 1.0},
+                   "separate_calls": kernels}
+        dom = "fused_moe_kernel"
     traffic = recorded_traffic(dom, wl.name)
     tokens = T * K * world
     value = job_rate(T * K, world, total_ms)
@@ -465,6 +490,8 @@ def run_ours(args, rank, world, local_rank):
     # stack's RMSNorm, and the layer call's x digit-record launch for up to 8 tokens
     launches_per_step = NL * ((1 if T <= 8 else 3) + 2 + (1 if stack else 0)
                               + (1 if args.api == "layer" and T <= 8 else 0))
+    if fused:
+        launches_per_step = 1 if stack else NL
 
     out = {
         "metric": METRIC,
@@ -479,15 +506,14 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "tokens_per_step": T, "layers": NL, "hidden": H,
-                   "intermediate": I,
-                   "experts": E, "top_k": k, "shared_experts": s.n_shared,
-                   "weights": "gs64 int4, fp16 scales", "activations": "fp32",
-                   "l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
+        "config": workload_config(wl),
+        "method": {"l2": "flushed before every step (2x L2 write, then 2x L2 read of another buffer), outside the timed intervals",
                    "timing": "CUDA graphs of up to 128 steps; events around each step (the value); "
                              "per-kernel figures from a second pass with events around each launch "
                              "(separate route_union / gate_up / down calls)",
-                   "api": ("coli_moe_layer, one call per layer" if args.api == "layer"
+                   "api": (("coli_moe_stack, one call (one launch) per step" if stack and fused else
+                            "coli_moe_layer, one call per layer" + (" (one fused launch)" if fused else ""))
+                           if args.api == "layer"
                            else "coli_moe_route_union + coli_moe_gate_up + coli_moe_down"),
                    "token_pool": R, "parallelism": f"replicas x{world}",
                    "mean_union_per_layer": float(nu.mean() / NL)},
@@ -507,10 +533,64 @@ def run_ours(args, rank, world, local_rank):
                       "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2],
                       "api": "coli_moe_layer with pinned-host x in and y out"}
     if stack:
-        out["config"]["kernel_figures"] = f"per step (sum over the {NL} layers' launches)"
+        out["method"]["kernel_figures"] = ("the step is one launch" if fused else
+                                           f"per step (sum over the {NL} layers' launches)")
+    if e2e and stack and fused:
+        out["e2e"]["api"] = "coli_moe_stack with pinned-host x in and y out"
+    if args.steady and not stack and fused:
+        out["steady_state"] = steady_state(args, B, dims, layers[0], s, xs, bufs, float(step_bytes.mean()), l2,
+                                           dev, peak)
     if world == 1 and not args.no_cpu_baseline and not stack:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     return out
+
+
+def steady_state(args, B, dims, L0, s, xs, bufs, call_bytes, l2, dev, peak):
+    """Back-to-back fused layer calls with no flush between them, each reading a different
+    copy of the layer's weights, the copies together at least 3x L2 of what the calls read,
+    so every call streams its experts from HBM while the calls follow each other as in a
+    decode loop."""
+    import math
+
+    import torch
+    C = max(2, math.ceil(3 * l2 / max(call_bytes, 1.0)))
+    copies = []
+    for c in range(C):
+        ex = L0["experts"].clone()
+        sh = L0["shared"].clone()
+        copies.append((ex, sh, B.make_weights(L0["wr"], L0["bias"], ex, sh, s.stride)))
+    T, R = xs[0].shape[0], len(xs)
+    n = 256
+
+    def call(i):
+        B.check(B.coli_moe_layer(dims, copies[i % C][2], xs[i % R], T, bufs.idx, bufs.w, None,
+                                 bufs.union_ids, bufs.n_union, bufs.offsets, bufs.assign, None, bufs.y,
+                                 bufs.ws), "coli_moe_layer")
+    for i in range(2 * C):
+        call(i)
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ev[0].record()
+        for i in range(n):
+            call(i)
+        ev[1].record()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    best = None
+    for _ in range(3):
+        g.replay()
+        torch.cuda.synchronize(dev)
+        ms = ev[0].elapsed_time(ev[1])
+        best = ms if best is None or ms < best else best
+    del g
+    per = best / n
+    gbs = call_bytes / (per * 1e-3) / 1e9
+    return {"ms_per_call": round(per, 6), "value": round(T / (per * 1e-3), 2), "unit": "tokens/s",
+            "gb_s": round(gbs, 1), "frac": round(gbs / peak, 4), "weight_copies": C,
+            "calls": n, "timing": "one CUDA graph of back-to-back calls, events at its two ends, "
+                                  "best of 3 replays; no L2 flush (each call reads another copy)"}
 
 
 def measured_tflops():
@@ -632,10 +712,9 @@ def run_prefill(args, wl, rank, world, dev):
         "ms_per_step": round(total_ms / K, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "tokens_per_step": T, "hidden": H, "intermediate": I,
-                   "experts": E, "top_k": k, "shared_experts": s.n_shared,
-                   "weights": "gs64 int4, fp16 scales, dequantised to bf16",
-                   "activations": "bf16", "l2": "flushed before every step, outside the timed intervals",
+        "config": workload_config(wl),
+        "method": {"weights": "gs64 int4, fp16 scales, dequantised to bf16",
+                   "l2": "flushed before every step, outside the timed intervals",
                    "parallelism": f"replicas x{world}", "n_union": int(bufs.n_union[0].item())},
         "roofline": {"bound": "tensor", "kernel": "grouped forward (gather + plan + 2 tcgen05 GEMM launches)",
                      "achieved": round(tflops, 1), "peak": burst,
@@ -686,20 +765,66 @@ def oracle_step(wl, wr, bias, x, blobs, shared):
     return oracle.forward_sparse(s.hidden, s.inter, s.top_k, s.n_shared, x, sub, shared, idx, w)
 
 
-def cpu_baseline(wl, seconds):
-    wr, bias, batches, blobs, shared = oracle_setup(wl, 4)
-    n = 0
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_rate(wl, seconds, threads, setup):
+    """Steps of the oracle done by `threads` threads in about `seconds` (the scalar C
+    oracle runs without the interpreter lock, so the threads run in parallel); every
+    thread finishes the step it is in."""
+    import threading
+    wr, bias, batches, blobs, shared = setup
+    counts = [0] * threads
+    deadline = time.perf_counter() + seconds
+
+    def work(j):
+        n = 0
+        while True:
+            oracle_step(wl, wr, bias, batches[(j + n) % len(batches)], blobs, shared)
+            n += 1
+            if time.perf_counter() >= deadline or n >= 64:
+                break
+        counts[j] = n
+
     t0 = time.perf_counter()
-    while True:
-        oracle_step(wl, wr, bias, batches[n % len(batches)], blobs, shared)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or n >= 64:
-            break
-    return {"value": round(n * wl.tokens / el, 4), "unit": "tokens/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{n} steps of {wl.tokens} token(s) of {wl.name} (route+union+forward, "
-                      f"scalar C, double accumulation, one thread), {el:.1f} s"}
+    ts = [threading.Thread(target=work, args=(j,)) for j in range(threads)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    el = time.perf_counter() - t0
+    return sum(counts), el
+
+
+def cpu_baseline(wl, seconds):
+    setup = oracle_setup(wl, 4)
+    n1, el1 = oracle_rate(wl, seconds / 3, 1, setup)
+    nth = os.cpu_count() or 1
+    nn, eln = oracle_rate(wl, 2 * seconds / 3, nth, setup)
+    return {"value": round(nn * wl.tokens / eln, 4), "unit": "tokens/s", "cores": nth,
+            "kind": "oracle", "cpu_model": cpu_model(),
+            "sample": f"{nn} steps of {wl.tokens} token(s) of {wl.name} on {nth} threads in {eln:.1f} s "
+                      "(route+union+forward, scalar C, double accumulation, one step per thread at a time)",
+            "one_thread": {"value": round(n1 * wl.tokens / el1, 4), "unit": "tokens/s", "cores": 1,
+                           "sample": f"{n1} steps in {el1:.1f} s"}}
+
+
+def workload_config(wl):
+    """The `config` object of a workload (shared by both arms)."""
+    s = wl.shape
+    return {"workload": wl.name, "tokens_per_step": wl.tokens, "layers": wl.layers, "hidden": s.hidden,
+            "intermediate": s.inter, "experts": s.n_experts, "top_k": s.top_k,
+            "shared_experts": s.n_shared, "weights": "gs64 int4, fp16 scales",
+            "activations": "bf16" if wl.x_dtype == "bf16" else "fp32"}
 
 
 def run_reference(args, rank):
@@ -728,7 +853,7 @@ def run_reference(args, rank):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el * 1e3 / done, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "tokens_per_step": wl.tokens},
+            "config": workload_config(wl),
             "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": 1,
                              "kind": "oracle",
                              "sample": f"{done} timed step(s) of {wl.tokens} token(s) "
@@ -736,6 +861,44 @@ def run_reference(args, rank):
                                        "rotating over 4 token batches"},
             "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+# The other configurations, each run by a short bench of its own (a subprocess, so that
+# each holds only its own weights): (workload, steps, extra flags)
+OTHER_CONFIGS = [
+    ("moe_h1024_i512_e64_k4_t1", 200, ["--steady"]),
+    ("moe_h1024_i512_e64_k4_t4_zipf", 200, ["--steady"]),
+    ("glm52_moe_h6144_i2048_e256_k8_t4_zipf", 100, []),
+    ("moe_h1024_i512_e64_k4_stack16_t1", 50, []),
+    ("glm52_stack16_h6144_i2048_e256_k8_t1", 20, []),
+    ("moe_h1024_i512_e64_k4_t2048_bf16_zipf", 20, []),
+    ("glm52_moe_h6144_i2048_e256_k8_t2048_bf16_zipf", 10, []),
+]
+
+
+def run_other_configs(args):
+    import subprocess
+    res = {}
+    for name, steps, extra in OTHER_CONFIGS:
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(steps),
+               "--warmup", "3", "--no-cpu-baseline", "--no-e2e", "--no-configs"] + extra
+        try:
+            p = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
+            line = [l for l in p.stdout.splitlines() if l.startswith("{")]
+            if p.returncode != 0 or not line:
+                res[name] = {"error": (p.stderr.strip().splitlines() or ["no output"])[-1][:300]}
+                continue
+            o = json.loads(line[-1])
+        except subprocess.TimeoutExpired:
+            res[name] = {"error": "timed out after 300 s"}
+            continue
+        r = {"value": o["value"], "unit": o["unit"], "ms_per_step": o["ms_per_step"], "steps": o["steps"],
+             "roofline": o.get("roofline"), "clocks": o.get("clocks")}
+        for key in ("step_hbm", "steady_state", "method"):
+            if key in o:
+                r[key] = o[key]
+        res[name] = r
+    return res
 
 
 def main():
@@ -761,6 +924,10 @@ def main():
         if world > 1:
             import torch
             torch.distributed.destroy_process_group()
+    if out is not None and world == 1 and not args.no_configs and args.workload == DEFAULT_WORKLOAD:
+        import torch
+        torch.cuda.empty_cache()
+        out["configs"] = run_other_configs(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 

@@ -195,13 +195,32 @@ COLI_API coli_status coli_moe_layer(const coli_moe_dims* dims, const coli_moe_we
  * h before reading it); calls whose GPU work overlaps (e.g. on two streams) race on it,
  * so serialise them.  The first call on a device sets up the array's device address
  * (once per device, with that device current): make that first call before any stream
- * capture.  Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+ * capture.  Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Device errors of a call (the status bits of coli_moe_read_status) are in the array's
+ * header until the next call on the device clears it: read them with
+ * coli_moe_noalloc_read_status before that.  A device reset (cudaDeviceReset, or a
+ * destroyed and re-created primary context) is not supported: the array's address is
+ * looked up once per device for the life of the process. */
 COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_dims* dims,
                                               const coli_moe_weights* weights, const float* x,
                                               int32_t T, const float* w, const int32_t* union_ids,
                                               const int32_t* n_union, const int32_t* offsets,
                                               const int32_t* assign, const float* residual,
                                               float* y, void* stream);
+
+/* Status word of the last coli_moe_forward_noalloc call on the current device (the
+ * allocation-free counterpart of coli_moe_read_status; synchronises `stream`, allocates
+ * nothing).  Returns COLI_OK, or COLI_EDEVICE / COLI_ETIMEOUT when bits are set; COLI_ECUDA
+ * if the array's address cannot be looked up. */
+COLI_API coli_status coli_moe_noalloc_read_status(uint32_t* status, void* stream);
+
+/* Diagnostic: run one bounded device wait that can only run out (an mbarrier nothing
+ * arrives at), with a budget of `budget_cycles` SM clock cycles (1 .. 2^32).  When the
+ * budget is spent the kernel records COLI_DEV_TIMEOUT and timeout site 99 in the workspace
+ * header (as every wait of the library does), writes 1 to the device int32 *returned and
+ * ends; the stream and context stay usable.  For tests of the failure path. */
+COLI_API coli_status coli_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t budget_cycles,
+                                             int32_t* returned, void* stream);
 
 /* Residual stack of decode layers, every layer resident in device memory:
  *   for l in 0 .. n_layers-1:  n = RMSNorm_l(x);  x = x + MoE_l(n);   y = x at the end,

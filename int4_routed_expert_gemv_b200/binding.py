@@ -26,7 +26,7 @@ EXPORTS = [
     "coli_moe_blob_bytes", "coli_moe_workspace_bytes", "coli_moe_workspace_init",
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
     "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_moe_stack", "coli_rmsnorm",
-    "coli_moe_forward_noalloc",
+    "coli_moe_forward_noalloc", "coli_moe_noalloc_read_status", "coli_debug_wait_timeout",
     "coli_status_string",
 ]
 
@@ -79,6 +79,8 @@ def lib():
                 "coli_moe_stack": (i32, [D, W, P, i32, ctypes.c_double, P, i32, P, P, P, sz, P]),
                 "coli_rmsnorm": (i32, [i32, i32, P, P, ctypes.c_double, P, P]),
                 "coli_moe_forward_noalloc": (i32, [D, W, P, i32, P, P, P, P, P, P, P, P]),
+                "coli_moe_noalloc_read_status": (i32, [ctypes.POINTER(ctypes.c_uint32), P]),
+                "coli_debug_wait_timeout": (i32, [P, sz, ctypes.c_uint64, P, P]),
                 "coli_status_string": (ctypes.c_char_p, [i32]),
             }
             for name, (res, args) in sig.items():
@@ -136,6 +138,16 @@ def coli_moe_workspace_bytes(dims: Dims, T_max: int) -> int:
 
 def coli_moe_workspace_init(ws: torch.Tensor, stream=None) -> int:
     return lib().coli_moe_workspace_init(_p(ws), ws.numel() * ws.element_size(), _s(stream))
+
+
+def coli_moe_noalloc_read_status(stream=None):
+    v = ctypes.c_uint32(0)
+    st = lib().coli_moe_noalloc_read_status(ctypes.byref(v), _s(stream))
+    return st, int(v.value)
+
+
+def coli_debug_wait_timeout(ws: torch.Tensor, budget_cycles: int, returned: torch.Tensor, stream=None) -> int:
+    return lib().coli_debug_wait_timeout(_p(ws), ws.numel(), int(budget_cycles), _p(returned), _s(stream))
 
 
 def coli_moe_read_status(ws: torch.Tensor, stream=None):

@@ -152,6 +152,15 @@ __device__ __forceinline__ void give_up(uint32_t* status, uint32_t site, volatil
     *dead = 1;
 }
 
+// The slow checks of a polling loop: whether any CTA has given up (a global read, an L2 round
+// trip) and whether this wait is over its budget.  A loop calls this once per poll, and
+// the checks run on every 1024th call only, so that a poll that succeeds is seen at once.
+__device__ __forceinline__ bool wait_expired(uint32_t& n, long long t0, uint32_t* status)
+{
+    if ((++n & 1023u) != 0u) return false;
+    return timed_out(status) || clock64() - t0 > kWaitBudgetCycles;
+}
+
 // Wait until *p >= target (acquire).  Bounded: after the budget, or once any CTA has timed
 // out, the CTA is marked dead and the wait returns false.
 __device__ __forceinline__ bool gwait(const uint32_t* p, uint32_t target, uint32_t* status, uint32_t site,
@@ -160,10 +169,11 @@ __device__ __forceinline__ bool gwait(const uint32_t* p, uint32_t target, uint32
     if (*dead) return false;
     if (ld_acquire(p) >= target) return true;
     const long long t0 = clock64();
+    uint32_t npoll = 0;
     while (true) {
         __nanosleep(128);   // polls leave the issue slots to the working warps
         if (ld_acquire(p) >= target) return true;
-        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+        if (wait_expired(npoll, t0, status)) {
             give_up(status, site, dead);
             return false;
         }
@@ -191,10 +201,11 @@ __device__ __forceinline__ bool mwait(uint64_t* bar, uint32_t parity, uint32_t* 
     if (mbar_try_wait(bar, parity)) return true;
     if (*dead) return false;
     const long long t0 = clock64();
+    uint32_t npoll = 0;
     while (true) {
         if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*dead) return false;
-        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+        if (wait_expired(npoll, t0, status)) {
             give_up(status, site, dead);
             return false;
         }
@@ -207,11 +218,12 @@ __device__ __forceinline__ bool swait(const int* p, int target, uint32_t* status
     const volatile int* vp = p;
     if (*vp >= target) return true;
     const long long t0 = clock64();
+    uint32_t npoll = 0;
     while (true) {
         __nanosleep(32);
         if (*vp >= target) return true;
         if (*dead) return false;
-        if (timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+        if (wait_expired(npoll, t0, status)) {
             give_up(status, site, dead);
             return false;
         }
@@ -354,6 +366,7 @@ __device__ __forceinline__ void build_tile(const void* row0, const void* row1, b
         if (HEP) {
             // (value, epoch) pairs, read until every pair carries this layer's epoch
             const long long t0 = clock64();
+            uint32_t npoll = 0;
             bool ok = false;
             while (!ok) {
                 ok = true;
@@ -369,7 +382,7 @@ __device__ __forceinline__ void build_tile(const void* row0, const void* row1, b
                     }
                 }
                 ok = __all_sync(0xffffffffu, ok);
-                if (!ok && (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles)) {
+                if (!ok && (*dead || wait_expired(npoll, t0, status))) {
                     if (lane == 0) give_up(status, 56, dead);
                     break;
                 }
@@ -564,6 +577,7 @@ __device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, 
     const bool mine = plane < 3 && (n >> 2) == (tq >> 1);
     float4 v[NP];
     const long long t0 = clock64();
+    uint32_t npoll = 0;
     bool ok = false;
     while (!ok) {
         ok = true;
@@ -576,7 +590,7 @@ __device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, 
                                 __uint_as_float(b.z));
         }
         ok = __all_sync(0xffffffffu, ok);
-        if (!ok && (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles)) {
+        if (!ok && (*dead || wait_expired(npoll, t0, status))) {
             if (lane == 0) give_up(status, 56, dead);
             break;
         }
@@ -625,12 +639,13 @@ __device__ __forceinline__ void digitize_h_row(const uint2* staged, const uint2*
         if (!ok) {
             const uint4* hp = reinterpret_cast<const uint4*>(row + 128 * pp + 4 * lane);
             const long long t0 = clock64();
+            uint32_t npoll = 0;
             while (true) {
                 a = __ldcg(hp);
                 b = __ldcg(hp + 1);
                 ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
                 if (ok) break;
-                if (*dead || timed_out(status) || clock64() - t0 > kWaitBudgetCycles) {
+                if (*dead || wait_expired(npoll, t0, status)) {
                     if (lane == 0) give_up(status, 56, dead);
                     break;
                 }
@@ -1144,6 +1159,7 @@ __device__ __forceinline__ void route_compute(const FusedParams& p, const Ctx& c
                 // whatever is there)
                 uint4 q[8];
                 const long long t0 = clock64();
+                uint32_t npoll = 0;
                 while (true) {
 #pragma unroll
                     for (int i = 0; i < 8; i++) {
@@ -1154,7 +1170,7 @@ __device__ __forceinline__ void route_compute(const FusedParams& p, const Ctx& c
 #pragma unroll
                     for (int i = 0; i < 8; i++) ok = ok && q[i].y == ep && q[i].w == ep;
                     if (dry || __all_sync(0xffffffffu, ok)) break;
-                    if (*c.dead || timed_out(p.status) || clock64() - t0 > kWaitBudgetCycles) {
+                    if (*c.dead || wait_expired(npoll, t0, p.status)) {
                         if (lane == 0) give_up(p.status, 41, c.dead);
                         break;
                     }

@@ -19,7 +19,11 @@
 //   * two calls whose work overlaps on the GPU (e.g. on two streams) race on the array;
 //     serialise them (one stream, or events);
 //   * the first call on a device looks up the array's device address (set-up, once per
-//     device, with that device current); make that first call before any stream capture.
+//     device, with that device current); make that first call before any stream capture;
+//   * the device status word of a call stays in the array's header until the next call
+//     clears it (coli_moe_noalloc_read_status reads it without allocating);
+//   * the looked-up address is kept for the life of the process: a device reset is not
+//     supported.
 #include <cuda_runtime.h>
 #include <mutex>
 #include <stdint.h>
@@ -129,4 +133,18 @@ extern "C" coli_status coli_moe_forward_noalloc(const coli_moe_dims* d, const co
     for (int mode = 0; mode < 2; mode++)
         if (coli::gemv_launch(mode, ps[mode], cs[mode], s) != cudaSuccess) return COLI_ECUDA;
     return COLI_OK;
+}
+
+extern "C" coli_status coli_moe_noalloc_read_status(uint32_t* status, void* stream)
+{
+    if (!status) return COLI_EINVAL;
+    DeviceScratch ds;
+    if (!scratch_for_current_device(ds)) return COLI_ECUDA;
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ds.addr, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return COLI_ECUDA;
+    *status = v;
+    if (v & COLI_DEV_TIMEOUT) return COLI_ETIMEOUT;
+    return v ? COLI_EDEVICE : COLI_OK;
 }

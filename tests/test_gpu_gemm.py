@@ -2,9 +2,11 @@
 bf16-weights mode: every weight bf16(q * scale), x bf16 as given, h exact, sums in double
 (the device carries h into the down projection as a bf16 hi + lo pair).
 
-Routing, union and assignment lists are checked bit for bit for every token; y on
-sampled tokens (the scalar oracle costs ~0.5 s per GLM-shaped token), within relative L2
-1e-4 and max 1e-3 rms.
+Routing, union and assignment lists are checked bit for bit for every token.  y, within
+relative L2 1e-4 and max 1e-3 rms: at hidden 1024 on every token; at the GLM shape (the
+scalar oracle costs ~0.5 s per token) on the first and last token of three experts of
+every group-size class (up to 16, 32, 64, 128 tokens and more, the token-box heights
+of the grouped GEMM), plus the batch's first and last token.
 """
 import numpy as np
 import pytest
@@ -47,15 +49,35 @@ def check_layer(L, x_bf16, T, sample, residual=None):
     return assert_y_close(y, y_ref)
 
 
+def group_edge_tokens(L, x_bf16, T):
+    """First and last token of three experts (lowest, middle, highest id) in every class
+    of token-group size, and the batch's first and last token."""
+    s = L.shape
+    idx, _, _ = oracle.route(x_bf16.float().numpy(), L.w_router_host, L.bias_host, s.top_k)
+    uid, nu, off, asg = oracle.union(idx, s.n_experts)
+    classes = {}
+    for u in range(nu):
+        c = off[u + 1] - off[u]
+        b = 0 if c <= 16 else 1 if c <= 32 else 2 if c <= 64 else 3 if c <= 128 else 4
+        classes.setdefault(b, []).append(u)
+    tokens = {0, T - 1}
+    for us in classes.values():
+        for u in {us[0], us[len(us) // 2], us[-1]}:
+            tokens.add(int(asg[off[u]]) // s.top_k)
+            tokens.add(int(asg[off[u + 1] - 1]) // s.top_k)
+    return sorted(tokens)
+
+
 @pytest.mark.parametrize("name", ["moe_h1024_i512_e64_k4_t2048_bf16_zipf",
                                   "glm52_moe_h6144_i2048_e256_k8_t2048_bf16_zipf"])
 def test_prefill_grouped_gemm(colimoe, name):
     wl = synth.WORKLOADS[name]
     L = make_device_layer(wl.shape, wl.seed, zipf=wl.zipf)
     x = synth.activations_bf16(wl.shape, wl.seed, wl.tokens, wl.x_variant)
-    rng = np.random.default_rng(7)
-    n_sample = 24 if wl.shape.hidden <= 1024 else 6
-    sample = [0, wl.tokens - 1] + rng.integers(0, wl.tokens, n_sample).tolist()
+    if wl.shape.hidden <= 1024:
+        sample = list(range(wl.tokens))
+    else:
+        sample = group_edge_tokens(L, x, wl.tokens)
     rel, mx = check_layer(L, x, wl.tokens, sample)
     print(f"{name}: rel L2 {rel:.2e}, max/rms {mx:.2e}")
 

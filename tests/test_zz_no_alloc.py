@@ -4,10 +4,13 @@ owns all device memory, or a latency-critical loop where cudaMalloc would synchr
 device).  Its scratch is a fixed array in the library's device memory instead of a
 caller-owned workspace.
 
-Checked through the C ABI against the regular coli_moe_forward on the same inputs, on two
-calls in a row (the array keeps the previous call's contents), within the parity
-tolerance of the other tests.  Collected last on purpose: a run that stops at the first
-failure has run every other test before this one.
+Checked through the C ABI, on two calls in a row (the array keeps the previous call's
+contents): against the oracle (same routing, y within the parity tolerance of the other
+tests) and against the regular coli_moe_forward; the device status word, read without
+allocating, stays clear after every call; a one-token call repeated after a four-token
+call (whose h is larger) gives the same y bit for bit, so no leftover contents are read.
+Collected last on purpose: a run that stops at the first failure has run every other
+test before this one.
 """
 import numpy as np
 import pytest
@@ -15,7 +18,7 @@ import torch
 
 from int4_routed_expert_gemv_b200 import binding as B
 from int4_routed_expert_gemv_b200 import synth
-from layers import assert_y_close, make_device_layer
+from layers import assert_y_close, make_device_layer, oracle_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +44,37 @@ def test_noalloc_forward_matches_regular_forward(colimoe, name):
         B.check(B.coli_moe_forward_noalloc(L.dims, L.weights, x, T, bufs.w, bufs.union_ids,
                                            bufs.n_union, bufs.offsets, bufs.assign, res, y),
                 "coli_moe_forward_noalloc")
+        assert B.coli_moe_noalloc_read_status() == (B.COLI_OK, 0)
         torch.cuda.synchronize()
-        assert_y_close(y.cpu().numpy(), y_ref.cpu().numpy())
-        outs.append(y.cpu().numpy())
+        y_h = y.cpu().numpy()
+        assert_y_close(y_h, y_ref.cpu().numpy())
+        # the oracle on the same input: routing identical, y within the parity bar
+        o = oracle_layer(L, x.cpu().numpy())
+        assert np.array_equal(bufs.idx[:T].cpu().numpy(), o["idx"])
+        assert_y_close(y_h, res.cpu().numpy() + o["y"])
+        outs.append(y_h)
     assert not np.array_equal(outs[0], outs[1])
+
+
+def test_noalloc_no_leftover_contents(colimoe):
+    """T = 1, then T = 4 (a larger h), then the T = 1 call again: identical y."""
+    wl = synth.WORKLOADS["moe_h1024_i512_e64_k4_t4_zipf"]
+    L = make_device_layer(wl.shape, wl.seed, zipf=wl.zipf)
+    ys = []
+    for T, variant in [(1, 51), (4, 52), (1, 51)]:
+        bufs = B.LayerBuffers(L.dims, T)
+        x = torch.from_numpy(synth.activations(wl.shape, wl.seed, T, variant)).cuda()
+        B.check(B.coli_moe_route_union(L.dims, L.w_router, L.bias, x, T, bufs.idx, bufs.w,
+                                       None, bufs.union_ids, bufs.n_union, bufs.offsets,
+                                       bufs.assign, bufs.ws))
+        y = torch.full((T, wl.shape.hidden), float("nan"), device="cuda")
+        B.check(B.coli_moe_forward_noalloc(L.dims, L.weights, x, T, bufs.w, bufs.union_ids,
+                                           bufs.n_union, bufs.offsets, bufs.assign, None, y),
+                "coli_moe_forward_noalloc")
+        assert B.coli_moe_noalloc_read_status() == (B.COLI_OK, 0)
+        ys.append(y.cpu().numpy())
+    assert np.isfinite(ys[1]).all()
+    assert np.array_equal(ys[0], ys[2])
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch(colimoe):
