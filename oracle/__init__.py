@@ -67,6 +67,18 @@ def lib():
             L.orc_forward.restype = i32
             L.orc_rmsnorm.argtypes = [i32, i32, P, P, dbl, P]
             L.orc_rmsnorm.restype = i32
+            L.orc_crumb.argtypes = [P, i64]
+            L.orc_crumb.restype = i32
+            L.orc_int8.argtypes = [P, i64]
+            L.orc_int8.restype = i32
+            L.orc_blob_bytes_fmt.argtypes = [i32, i32, i32]
+            L.orc_blob_bytes_fmt.restype = i64
+            L.orc_blob_weight_fmt.argtypes = [i32, i32, i32, P, i32, i64, i64]
+            L.orc_blob_weight_fmt.restype = dbl
+            L.orc_expert_fmt.argtypes = [i32, i32, i32, P, P, P]
+            L.orc_expert_fmt.restype = i32
+            L.orc_forward_fmt.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, i64, P, P, P, P]
+            L.orc_forward_fmt.restype = i32
             _lib = L
     return _lib
 
@@ -169,6 +181,55 @@ def forward(H, I, E, k, n_shared, x, experts, stride, shared, idx, w, bf16=False
     _check(lib().orc_forward(H, I, E, k, n_shared, T, _ptr(x), _ptr(experts), stride, _ptr(sh),
                              _ptr(idx), _ptr(w), int(bf16), _ptr(y)), "forward")
     return y
+
+
+# weight containers (orc_forward_fmt): gs64 int4, gs64 int8, per-row int4, gs64 int2
+FMT_INT4_G64, FMT_INT8_G64, FMT_INT4_ROW, FMT_INT2_G64 = 0, 1, 2, 3
+
+
+def crumb(row: np.ndarray, c: int) -> int:
+    row = _c(row, np.uint8)
+    return lib().orc_crumb(_ptr(row), c)
+
+
+def int8_value(row: np.ndarray, c: int) -> int:
+    row = _c(row, np.uint8)
+    return lib().orc_int8(_ptr(row), c)
+
+
+def blob_bytes_fmt(H: int, I: int, fmt: int) -> int:
+    return lib().orc_blob_bytes_fmt(H, I, fmt)
+
+
+def blob_weight_fmt(H, I, fmt, blob, which, r, c) -> float:
+    blob = _c(blob, np.uint8)
+    return lib().orc_blob_weight_fmt(H, I, fmt, _ptr(blob), which, r, c)
+
+
+def forward_fmt(H, I, E, k, n_shared, fmt, x, experts, stride, shared, idx, w):
+    """y [T][H] float32 for blobs in container fmt (fp32 contract)."""
+    x = _c(x, np.float32)
+    T = x.shape[0]
+    experts = _c(experts, np.uint8)
+    sh = None if shared is None else _c(shared, np.uint8)
+    idx = _c(idx, np.int32)
+    w = _c(w, np.float32)
+    y = np.zeros((T, H), np.float32)
+    _check(lib().orc_forward_fmt(H, I, E, k, n_shared, T, fmt, _ptr(x), _ptr(experts), stride, _ptr(sh),
+                                 _ptr(idx), _ptr(w), _ptr(y)), "forward_fmt")
+    return y
+
+
+def forward_sparse_fmt(H, I, k, n_shared, fmt, x, blobs: dict, shared, idx, w):
+    """forward_fmt for tokens whose experts are given as a dict {expert_id: blob}."""
+    ids = sorted(blobs)
+    remap = {e: j for j, e in enumerate(ids)}
+    nb = len(blobs[ids[0]])
+    packed = np.zeros((len(ids), nb), np.uint8)
+    for j, e in enumerate(ids):
+        packed[j] = np.asarray(blobs[e], np.uint8)
+    idx2 = np.vectorize(lambda e: remap[int(e)])(np.asarray(idx)).astype(np.int32)
+    return forward_fmt(H, I, len(ids), k, n_shared, fmt, x, packed, nb, shared, idx2, w)
 
 
 def forward_sparse(H, I, k, n_shared, x, blobs: dict, shared, idx, w, bf16=False):

@@ -381,3 +381,159 @@ int orc_rmsnorm(int H, int T, const float *x, const float *gamma, double eps, fl
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Other weight containers                                                               */
+/* ------------------------------------------------------------------------------------ */
+/* The engine's kernels also come in int8 and packed int2 forms, and the older per-row
+ * int4 container predates gs64 (colibri README.zh-CN, "开始使用 / 2. 获取模型"; the
+ * technical article's "精度与语义" section; the nxmr essay on the hand-written quantised
+ * kernels).  The pages fix no layout for these.  The readings taken here keep the gs64
+ * blob's order of matrices and change only the payload and the scale axis:
+ *   fmt 0  int4, one fp16 scale per 64 input columns (the gs64 container above);
+ *   fmt 1  int8 two's complement [-128, 127], one byte per weight, gs64 fp16 scales;
+ *   fmt 2  int4 nibbles as in fmt 0, one fp16 scale per row ("per-row");
+ *   fmt 3  int2 two's complement [-2, 1], four per byte with the lowest-index column in
+ *          the lowest two bits, gs64 fp16 scales.
+ * Blob: Gq [I][H*b/8] | Uq [I][H*b/8] | Dq [H][I*b/8] | Gs | Us | Ds, b the payload bits;
+ * the scale blocks are [rows][in/64] fp16 (fmt 0, 1, 3) or [rows] fp16 (fmt 2).
+ * Only the fp32 contract (mode 0) is defined for them. */
+
+/* Signed 2-bit value of column c in a packed row (two's complement, lowest bits first). */
+int orc_crumb(const uint8_t *row, int64_t c)
+{
+    int v = (row[c >> 2] >> (2 * (int)(c & 3))) & 3;
+    return v >= 2 ? v - 4 : v;
+}
+
+/* Signed 8-bit value of column c. */
+int orc_int8(const uint8_t *row, int64_t c)
+{
+    int v = row[c];
+    return v >= 128 ? v - 256 : v;
+}
+
+static int fmt_bits(int fmt) { return fmt == 1 ? 8 : fmt == 3 ? 2 : 4; }
+static int fmt_valid(int fmt) { return fmt >= 0 && fmt <= 3; }
+/* fp16 scales per row of a matrix with `in_dim` input columns */
+static int64_t fmt_scales_per_row(int fmt, int64_t in_dim) { return fmt == 2 ? 1 : in_dim / 64; }
+
+int64_t orc_blob_bytes_fmt(int H, int I, int fmt)
+{
+    if (!fmt_valid(fmt))
+        return -1;
+    int64_t h = H, i = I, b = fmt_bits(fmt);
+    int64_t payload = 3 * (h * i * b / 8);
+    int64_t scales = 2 * i * fmt_scales_per_row(fmt, h) * 2 + h * fmt_scales_per_row(fmt, i) * 2;
+    return payload + scales;
+}
+
+typedef struct {
+    const uint8_t *gq, *uq, *dq;
+    const uint16_t *gs, *us, *ds;
+} orc_fmt_view;
+
+static orc_fmt_view view_blob_fmt(int H, int I, int fmt, const uint8_t *blob)
+{
+    int64_t h = H, i = I, b = fmt_bits(fmt);
+    orc_fmt_view v;
+    v.gq = blob;
+    v.uq = blob + i * h * b / 8;
+    v.dq = blob + 2 * (i * h * b / 8);
+    const uint8_t *s = blob + 3 * (i * h * b / 8);
+    v.gs = (const uint16_t *)s;
+    v.us = (const uint16_t *)(s + i * fmt_scales_per_row(fmt, h) * 2);
+    v.ds = (const uint16_t *)(s + 2 * i * fmt_scales_per_row(fmt, h) * 2);
+    return v;
+}
+
+/* Dequantised weight (r, c) of a [rows][in_dim] matrix in container fmt: q * scale. */
+static double weight_fmt(int fmt, const uint8_t *q, const uint16_t *s, int64_t in_dim, int64_t r,
+                         int64_t c)
+{
+    int64_t row_bytes = in_dim * fmt_bits(fmt) / 8;
+    const uint8_t *row = q + r * row_bytes;
+    int qv = fmt == 1 ? orc_int8(row, c) : fmt == 3 ? orc_crumb(row, c) : orc_nibble(row, c);
+    double sc = fmt == 2 ? orc_half(s[r]) : orc_half(s[r * (in_dim / 64) + c / 64]);
+    return (double)qv * sc;   /* exact: at most 8 bits times 11 bits */
+}
+
+double orc_blob_weight_fmt(int H, int I, int fmt, const uint8_t *blob, int which, int64_t r, int64_t c)
+{
+    orc_fmt_view v = view_blob_fmt(H, I, fmt, blob);
+    if (which == 0)
+        return weight_fmt(fmt, v.gq, v.gs, H, r, c);
+    if (which == 1)
+        return weight_fmt(fmt, v.uq, v.us, H, r, c);
+    return weight_fmt(fmt, v.dq, v.ds, I, r, c);
+}
+
+/* One expert on one token in container fmt (fp32 contract): as orc_expert. */
+int orc_expert_fmt(int H, int I, int fmt, const uint8_t *blob, const float *x, double *out)
+{
+    if (H <= 0 || I <= 0 || H % 64 || I % 64 || !fmt_valid(fmt))
+        return ORC_EINVAL;
+    orc_fmt_view v = view_blob_fmt(H, I, fmt, blob);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!h)
+        return ORC_ENOMEM;
+    for (int64_t i = 0; i < I; i++) {
+        double g = 0.0, u = 0.0;
+        for (int64_t c = 0; c < H; c++)
+            g += weight_fmt(fmt, v.gq, v.gs, H, i, c) * (double)x[c];
+        for (int64_t c = 0; c < H; c++)
+            u += weight_fmt(fmt, v.uq, v.us, H, i, c) * (double)x[c];
+        h[i] = silu(g) * u;
+    }
+    for (int64_t r = 0; r < H; r++) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < I; i++)
+            acc += weight_fmt(fmt, v.dq, v.ds, I, r, i) * h[i];
+        out[r] = acc;
+    }
+    free(h);
+    return ORC_OK;
+}
+
+/* The layer of orc_forward (fp32 contract) with every blob in container fmt. */
+int orc_forward_fmt(int H, int I, int E, int k, int n_shared, int T, int fmt, const float *x,
+                    const uint8_t *experts, int64_t stride, const uint8_t *shared,
+                    const int32_t *idx, const float *w, float *y)
+{
+    if (H <= 0 || I <= 0 || H % 64 || I % 64 || E <= 0 || k < 1 || k > E || T < 0 ||
+        (n_shared != 0 && n_shared != 1) || (n_shared == 1 && !shared) || !fmt_valid(fmt))
+        return ORC_EINVAL;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)H);
+    double *ye = (double *)malloc(sizeof(double) * (size_t)H);
+    if (!acc || !ye) {
+        free(acc);
+        free(ye);
+        return ORC_ENOMEM;
+    }
+    int rc = ORC_OK;
+    for (int64_t t = 0; t < T && rc == ORC_OK; t++) {
+        const float *xt = x + t * H;
+        for (int64_t r = 0; r < H; r++)
+            acc[r] = 0.0;
+        if (n_shared) {
+            rc = orc_expert_fmt(H, I, fmt, shared, xt, ye);
+            for (int64_t r = 0; r < H && rc == ORC_OK; r++)
+                acc[r] += ye[r];
+        }
+        for (int s = 0; s < k && rc == ORC_OK; s++) {
+            int32_t e = idx[t * k + s];
+            if (e < 0 || e >= E) {
+                rc = ORC_EINVAL;
+                break;
+            }
+            rc = orc_expert_fmt(H, I, fmt, experts + (int64_t)e * stride, xt, ye);
+            for (int64_t r = 0; r < H && rc == ORC_OK; r++)
+                acc[r] += (double)w[t * k + s] * ye[r];
+        }
+        for (int64_t r = 0; r < H; r++)
+            y[t * H + r] = (float)acc[r];
+    }
+    free(acc);
+    free(ye);
+    return rc;
+}
