@@ -214,6 +214,36 @@ COLI_API coli_status coli_moe_forward_noalloc(const coli_moe_dims* dims,
  * if the array's address cannot be looked up. */
 COLI_API coli_status coli_moe_noalloc_read_status(uint32_t* status, void* stream);
 
+/* Other weight containers (the engine's int8 and packed int2 kernels, and the older
+ * per-row int4 container; colibri README.zh-CN "开始使用 / 2. 获取模型", the technical
+ * article's "精度与语义").  The blob keeps the gs64 order Gq | Uq | Dq | Gs | Us | Ds and
+ * changes the payload or the scale axis:
+ *   COLI_FMT_INT4_G64  int4 nibbles, fp16 scale per 64 input columns (the gs64 blob);
+ *   COLI_FMT_INT8_G64  int8 two's complement, one byte per weight, gs64 fp16 scales;
+ *   COLI_FMT_INT4_ROW  int4 nibbles, one fp16 scale per row;
+ *   COLI_FMT_INT2_G64  int2 two's complement in [-2, 1], four per byte, lowest-index
+ *                      column in the lowest bits, gs64 fp16 scales.
+ * q matrices are [rows][in * b / 8] bytes; scale blocks [rows][in / 64] (or [rows]) fp16. */
+#define COLI_FMT_INT4_G64 0
+#define COLI_FMT_INT8_G64 1
+#define COLI_FMT_INT4_ROW 2
+#define COLI_FMT_INT2_G64 3
+
+/* Bytes of one expert blob in container fmt (0 for invalid arguments). */
+COLI_API size_t coli_moe_blob_bytes_fmt(int32_t hidden, int32_t inter, int32_t fmt);
+
+/* Decode forward (fp32 activations, 1 <= T <= 4) for blobs in container fmt: arguments and
+ * result as coli_moe_forward with dtype COLI_F32 (idx is not needed: the union lists and w
+ * carry the routing); expert_stride >= coli_moe_blob_bytes_fmt, a multiple of 256.  Two
+ * launches (gate/up + SwiGLU, then down + combine); y's sums run in one fixed order.
+ * T > 4 returns COLI_EUNSUPPORTED. */
+COLI_API coli_status coli_moe_forward_fmt(const coli_moe_dims* dims, int32_t fmt,
+                                          const coli_moe_weights* weights, const float* x, int32_t T,
+                                          const float* w, const int32_t* union_ids,
+                                          const int32_t* n_union, const int32_t* offsets,
+                                          const int32_t* assign, const float* residual, float* y,
+                                          void* ws, size_t ws_bytes, void* stream);
+
 /* Diagnostic: run one bounded device wait that can only run out (an mbarrier nothing
  * arrives at), with a budget of `budget_cycles` SM clock cycles (1 .. 2^32).  When the
  * budget is spent the kernel records COLI_DEV_TIMEOUT and timeout site 99 in the workspace

@@ -27,6 +27,7 @@ EXPORTS = [
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
     "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_moe_stack", "coli_rmsnorm",
     "coli_moe_forward_noalloc", "coli_moe_noalloc_read_status", "coli_debug_wait_timeout",
+    "coli_moe_blob_bytes_fmt", "coli_moe_forward_fmt",
     "coli_status_string",
 ]
 
@@ -81,6 +82,8 @@ def lib():
                 "coli_moe_forward_noalloc": (i32, [D, W, P, i32, P, P, P, P, P, P, P, P]),
                 "coli_moe_noalloc_read_status": (i32, [ctypes.POINTER(ctypes.c_uint32), P]),
                 "coli_debug_wait_timeout": (i32, [P, sz, ctypes.c_uint64, P, P]),
+                "coli_moe_blob_bytes_fmt": (sz, [i32, i32, i32]),
+                "coli_moe_forward_fmt": (i32, [D, i32, W, P, i32, P, P, P, P, P, P, P, P, sz, P]),
                 "coli_status_string": (ctypes.c_char_p, [i32]),
             }
             for name, (res, args) in sig.items():
@@ -138,6 +141,20 @@ def coli_moe_workspace_bytes(dims: Dims, T_max: int) -> int:
 
 def coli_moe_workspace_init(ws: torch.Tensor, stream=None) -> int:
     return lib().coli_moe_workspace_init(_p(ws), ws.numel() * ws.element_size(), _s(stream))
+
+
+FMT_INT4_G64, FMT_INT8_G64, FMT_INT4_ROW, FMT_INT2_G64 = 0, 1, 2, 3
+
+
+def coli_moe_blob_bytes_fmt(hidden: int, inter: int, fmt: int) -> int:
+    return int(lib().coli_moe_blob_bytes_fmt(hidden, inter, fmt))
+
+
+def coli_moe_forward_fmt(dims, fmt, weights, x, T, w, union_ids, n_union, offsets, assign, residual, y, ws,
+                         stream=None) -> int:
+    return lib().coli_moe_forward_fmt(ctypes.byref(dims), int(fmt), ctypes.byref(weights), _p(x), T, _p(w),
+                                      _p(union_ids), _p(n_union), _p(offsets), _p(assign), _p(residual), _p(y),
+                                      _p(ws), ws.numel(), _s(stream))
 
 
 def coli_moe_noalloc_read_status(stream=None):

@@ -7,6 +7,7 @@
 #include "../../include/colimoe.h"
 #include "common.cuh"
 #include "fused.cuh"
+#include "fmt.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
 #include "rmsnorm.cuh"
@@ -566,3 +567,57 @@ const char* coli_status_string(coli_status s)
 }
 
 }  // extern "C"
+
+size_t coli_moe_blob_bytes_fmt(int32_t hidden, int32_t inter, int32_t fmt)
+{
+    if (hidden < 64 || inter < 64 || hidden % 64 || inter % 64) return 0;
+    return fmt_blob_bytes(hidden, inter, fmt);
+}
+
+coli_status coli_moe_forward_fmt(const coli_moe_dims* dims, int32_t fmt, const coli_moe_weights* weights,
+                                 const float* x, int32_t T, const float* w, const int32_t* union_ids,
+                                 const int32_t* n_union, const int32_t* offsets, const int32_t* assign,
+                                 const float* residual, float* y, void* ws, size_t ws_bytes, void* stream)
+{
+    if (!dims_ok(dims) || T < 0 || fmt < 0 || fmt > 3) return COLI_EINVAL;
+    if (T == 0) return COLI_OK;
+    if (T > kFmtMaxT) return COLI_EUNSUPPORTED;
+    const size_t blob = fmt_blob_bytes(dims->hidden, dims->inter, fmt);
+    if (!weights || !weights->experts || !aligned16(weights->experts) ||
+        (dims->n_shared && (!weights->shared || !aligned16(weights->shared))) ||
+        weights->expert_stride < blob || weights->expert_stride % 256 || !x || !aligned16(x) || !w ||
+        !union_ids || !n_union || !offsets || !assign || !y || !aligned16(y) ||
+        (residual && !aligned16(residual)))
+        return COLI_EINVAL;
+    coli_status st = ws_check(dims, T, ws, ws_bytes);
+    if (st != COLI_OK) return st;
+    DevInfo di;
+    if (!dev_info(di)) return COLI_ECUDA;
+    // x of the batch and one segment's h in shared memory
+    if ((size_t)T * dims->hidden * 4 > di.smem_optin || (size_t)T * dims->inter * 4 > di.smem_optin)
+        return COLI_EUNSUPPORTED;
+    const WsLayout W = ws_layout(dims, T);
+    FmtParams f;
+    memset(&f, 0, sizeof(f));
+    f.H = dims->hidden;
+    f.I = dims->inter;
+    f.E = dims->n_experts;
+    f.k = dims->top_k;
+    f.T = T;
+    f.n_shared = dims->n_shared;
+    f.fmt = fmt;
+    f.experts = weights->experts;
+    f.stride = weights->expert_stride;
+    f.shared = weights->shared;
+    f.x = x;
+    f.w = w;
+    f.union_ids = union_ids;
+    f.n_union = n_union;
+    f.offsets = offsets;
+    f.assign = assign;
+    f.h = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.h);
+    f.residual = residual;
+    f.y = y;
+    f.status = reinterpret_cast<uint32_t*>(ws);
+    return cuda_status(fmt_forward_launch(f, di.sms, (cudaStream_t)stream));
+}
