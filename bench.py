@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--steady", action="store_true",
                     help="also time back-to-back calls (no flush) rotating over weight copies "
                          "that together hold at least 3x L2")
+    ap.add_argument("--formats-only", action="store_true",
+                    help="print only the weight-container comparison (int4 gs64 / int8 gs64 / int4 per-row / "
+                         "int2 gs64): speed at the GLM shape and error against fp32 weights at hidden 1024")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other configurations' lines (run by default at N=1)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -876,6 +879,121 @@ OTHER_CONFIGS = [
 ]
 
 
+def run_formats(args):
+    """The weight containers side by side.  Speed: the GLM-shaped layer (hidden 6144, 256
+    experts, top-8 + shared), one token, random payloads, coli_moe_forward_fmt timed in
+    CUDA graphs with an L2 flush before every call.  Accuracy: the hidden-1024 layer with
+    fp32 weights N(0, 0.05) quantised by the package's host quantiser, y of the GPU path
+    against the same layer with the unquantised weights (numpy, double)."""
+    import torch
+
+    from int4_routed_expert_gemv_b200 import binding as B
+    from int4_routed_expert_gemv_b200 import build as builder
+    from int4_routed_expert_gemv_b200 import quantize as Q
+    from int4_routed_expert_gemv_b200 import synth
+    builder.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    names = {0: "int4_gs64", 1: "int8_gs64", 2: "int4_per_row", 3: "int2_gs64"}
+    peak, peak_kind = measured_peaks()
+    out = {}
+    # speed at the GLM shape
+    s = synth.GLM
+    H, I, E, k = s.hidden, s.inter, s.n_experts, s.top_k
+    dims = B.make_dims(H, I, E, k, 1)
+    wr = torch.from_numpy(synth.router_weight(s, 1)).to(dev)
+    R = 16
+    xs = [torch.from_numpy(synth.activations(s, 1, 1, 2000 + i)).to(dev) for i in range(R)]
+    routes = []
+    for i in range(R):
+        b = B.LayerBuffers(dims, 1, device=dev)
+        B.check(B.coli_moe_route_union(dims, wr, None, xs[i], 1, b.idx, b.w, None, b.union_ids, b.n_union,
+                                       b.offsets, b.assign, b.ws))
+        routes.append(b)
+    torch.cuda.synchronize(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    y = torch.empty(1, H, device=dev)
+    K = min(args.steps, 100)
+    for fmt in range(4):
+        bb = B.coli_moe_blob_bytes_fmt(H, I, fmt)
+        stride = (bb + 255) // 256 * 256
+        qb = 3 * H * I * Q.BITS[fmt] // 8
+        ex = torch.randint(0, 256, (E + 1, stride), dtype=torch.uint8, device=dev)
+        ex[:, qb:bb].view(torch.float16).fill_(0.01)
+        wts = B.make_weights(wr, None, ex[:E].reshape(-1), ex[E], stride)
+        def call(i):
+            b = routes[i % R]
+            B.check(B.coli_moe_forward_fmt(dims, fmt, wts, xs[i % R], 1, b.w, b.union_ids, b.n_union, b.offsets,
+                                           b.assign, None, y, b.ws))
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize(dev)
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(K)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(K):
+                flush_buf.zero_()
+                evs[i][0].record()
+                call(i)
+                evs[i][1].record()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+        del g
+        nb = float(np.mean([int(routes[i % R].n_union[0].item()) for i in range(K)]))
+        step_bytes = (nb + 1) * bb + E * H * 0
+        gbs = step_bytes / (ms * 1e-3) / 1e9
+        out[names[fmt]] = {"blob_bytes_glm": bb, "bits_per_weight": round(8.0 * bb / (3 * H * I), 4),
+                           "glm_t1": {"us_per_call": round(ms * 1e3, 2), "expert_bytes": step_bytes,
+                                      "gb_s": round(gbs, 1), "frac": round(gbs / peak, 4)}}
+        del ex
+    # accuracy at hidden 1024 against fp32 weights
+    s1 = synth.LayerShape(1024, 512, 64, 4, 1)
+    H1, I1, E1, k1 = s1.hidden, s1.inter, s1.n_experts, s1.top_k
+    rng = np.random.default_rng(12)
+    Wf = [[(rng.standard_normal(shp) * 0.05).astype(np.float32) for shp in ((I1, H1), (I1, H1), (H1, I1))]
+          for _ in range(E1 + 1)]
+    dims1 = B.make_dims(H1, I1, E1, k1, 1)
+    wr1_h = synth.router_weight(s1, 0)
+    wr1 = torch.from_numpy(wr1_h).to(dev)
+    T1 = 4
+    x1_h = synth.activations(s1, 0, T1, 300)
+    x1 = torch.from_numpy(x1_h).to(dev)
+    b1 = B.LayerBuffers(dims1, T1, device=dev)
+    B.check(B.coli_moe_route_union(dims1, wr1, None, x1, T1, b1.idx, b1.w, None, b1.union_ids, b1.n_union,
+                                   b1.offsets, b1.assign, b1.ws))
+    idx = b1.idx[:T1].cpu().numpy()
+    wgt = b1.w[:T1].cpu().numpy().astype(np.float64)
+
+    def expert64(G, U, D, xt):
+        g = G.astype(np.float64) @ xt
+        u = U.astype(np.float64) @ xt
+        return D.astype(np.float64) @ (g / (1.0 + np.exp(-g)) * u)
+    y32 = np.zeros((T1, H1))
+    for t in range(T1):
+        xt = x1_h[t].astype(np.float64)
+        y32[t] = expert64(*Wf[E1], xt) + sum(wgt[t, j] * expert64(*Wf[idx[t, j]], xt) for j in range(k1))
+    for fmt in range(4):
+        bb = B.coli_moe_blob_bytes_fmt(H1, I1, fmt)
+        stride = (bb + 255) // 256 * 256
+        host = np.zeros((E1 + 1, stride), np.uint8)
+        for e in range(E1 + 1):
+            host[e, :bb] = Q.expert_blob(*Wf[e], fmt)[0]
+        ex = torch.from_numpy(host).to(dev)
+        wts = B.make_weights(wr1, None, ex[:E1].reshape(-1), ex[E1], stride)
+        y1 = torch.empty(T1, H1, device=dev)
+        B.check(B.coli_moe_forward_fmt(dims1, fmt, wts, x1, T1, b1.w, b1.union_ids, b1.n_union, b1.offsets,
+                                       b1.assign, None, y1, b1.ws))
+        yq = y1.cpu().numpy().astype(np.float64)
+        out[names[fmt]]["h1024_t4_rel_l2_vs_fp32_weights"] = float(
+            np.linalg.norm(yq - y32) / np.linalg.norm(y32))
+    return {"formats": out, "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
+            "method": "speed: coli_moe_forward_fmt (two launches), GLM shape, T=1, random payloads, "
+                      f"CUDA graph of {K} calls with an L2 flush before each; accuracy: hidden 1024, T=4, "
+                      "fp32 weights N(0, 0.05) quantised by quantize.py, vs the fp32-weight layer in double"}
+
+
 def run_other_configs(args):
     import subprocess
     res = {}
@@ -898,6 +1016,15 @@ def run_other_configs(args):
             if key in o:
                 r[key] = o[key]
         res[name] = r
+    # the weight containers (a bench of their own)
+    cmd = [sys.executable, os.path.abspath(__file__), "--formats-only", "--steps", "100"]
+    try:
+        p = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
+        line = [l for l in p.stdout.splitlines() if l.startswith("{")]
+        res["weight_containers"] = json.loads(line[-1]) if p.returncode == 0 and line else \
+            {"error": (p.stderr.strip().splitlines() or ["no output"])[-1][:300]}
+    except subprocess.TimeoutExpired:
+        res["weight_containers"] = {"error": "timed out after 300 s"}
     return res
 
 
@@ -910,6 +1037,9 @@ def main():
         out = run_reference(args, rank)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+    if args.formats_only:
+        print(json.dumps(run_formats(args)), flush=True)
         return
     if world > 1:
         import datetime

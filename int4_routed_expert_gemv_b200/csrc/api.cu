@@ -594,7 +594,7 @@ coli_status coli_moe_forward_fmt(const coli_moe_dims* dims, int32_t fmt, const c
     DevInfo di;
     if (!dev_info(di)) return COLI_ECUDA;
     // x of the batch and one segment's h in shared memory
-    if ((size_t)T * dims->hidden * 4 > di.smem_optin || (size_t)T * dims->inter * 4 > di.smem_optin)
+    if ((size_t)T * dims->hidden * 5 > di.smem_optin || (size_t)T * dims->inter * 5 > di.smem_optin)
         return COLI_EUNSUPPORTED;
     const WsLayout W = ws_layout(dims, T);
     FmtParams f;

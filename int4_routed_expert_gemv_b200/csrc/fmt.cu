@@ -32,7 +32,14 @@ struct Fmt {
     static constexpr int per_word = 32 / bits;      // values in a 32-bit word
     static constexpr int per_chunk = 4 * per_word;  // values in a 16-byte chunk
     static constexpr bool per_row = FMT == FMT_INT4_ROW;
+    // activations in shared memory: the per_chunk values of a chunk, then 4 floats of
+    // padding, so that the lanes (one chunk each) read 16 bytes from distinct banks
+    static constexpr int pad_chunk = per_chunk + 4;
 };
+
+// floats of one activation row of `n` values in the padded layout
+template <int FMT>
+__host__ __device__ constexpr int padded_row(int n) { return n / Fmt<FMT>::per_chunk * Fmt<FMT>::pad_chunk; }
 
 __host__ __device__ inline int fmt_bits(int fmt) { return fmt == FMT_INT8_G64 ? 8 : fmt == FMT_INT2_G64 ? 2 : 4; }
 __host__ __device__ inline int64_t scales_per_row(int fmt, int64_t in_dim) { return fmt == FMT_INT4_ROW ? 1 : in_dim / 64; }
@@ -54,33 +61,62 @@ __host__ __device__ inline FmtBlob fmt_blob(int H, int I, int fmt)
     return b;
 }
 
-// value j (0 <= j < per_word) of a word, sign-extended
+// value j (0 <= j < per_word) of a word as a float: the field read as an offset-binary
+// code (two's complement with the sign bit flipped) inside the mantissa of 2^23, minus
+// 2^23 and the offset (exact; full-rate integer and float operations only)
 template <int FMT>
-__device__ __forceinline__ int field(uint32_t w, int j)
+__device__ __forceinline__ float field_f(uint32_t w, int j)
 {
     constexpr int b = Fmt<FMT>::bits;
-    return (int)(w << (32 - b * (j + 1))) >> (32 - b);
+    constexpr uint32_t mask = (1u << b) - 1u, sign = 1u << (b - 1);
+    const uint32_t u = ((w >> (b * j)) & mask) ^ (sign | 0x4B000000u);
+    return __uint_as_float(u) - (8388608.0f + (float)sign);
 }
 
-// sum_j q_j * xv_j over one 16-byte chunk for up to kFmtMaxT token rows of x (shared
-// memory, consecutive columns starting at col)
+// sum_v q_v * act_v over one 16-byte chunk, for up to kFmtMaxT activation rows (padded
+// layout in shared memory; row r of chunk ch at act + r * row_floats + ch * pad_chunk)
 template <int FMT>
-__device__ __forceinline__ void chunk_dot(const uint4& wv, const float* xs, int H, int col, int cnt,
+__device__ __forceinline__ void chunk_dot(const uint4& wv, const float* act, int row_floats, int ch, int cnt,
                                           const int (&tok)[kFmtMaxT], float (&acc)[kFmtMaxT])
 {
     const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int m = 0; m < kFmtMaxT; m++) {
-        if (m < cnt) {
-            const float* xr = xs + (size_t)tok[m] * H + col;
-            float a = 0.0f;
+    for (int wi = 0; wi < 4; wi++) {
+        float v[Fmt<FMT>::per_word];
 #pragma unroll
-            for (int wi = 0; wi < 4; wi++)
+        for (int j = 0; j < Fmt<FMT>::per_word; j++) v[j] = field_f<FMT>(words[wi], j);
 #pragma unroll
-                for (int j = 0; j < Fmt<FMT>::per_word; j++)
-                    a = fmaf((float)field<FMT>(words[wi], j), xr[wi * Fmt<FMT>::per_word + j], a);
-            acc[m] += a;
+        for (int m = 0; m < kFmtMaxT; m++) {
+            if (m < cnt) {
+                const float4* xr = reinterpret_cast<const float4*>(act + (size_t)tok[m] * row_floats +
+                                                                    ch * Fmt<FMT>::pad_chunk + wi * Fmt<FMT>::per_word);
+                float a = acc[m];
+#pragma unroll
+                for (int q = 0; q < Fmt<FMT>::per_word / 4; q++) {
+                    const float4 x4 = xr[q];
+                    a = fmaf(v[4 * q], x4.x, a);
+                    a = fmaf(v[4 * q + 1], x4.y, a);
+                    a = fmaf(v[4 * q + 2], x4.z, a);
+                    a = fmaf(v[4 * q + 3], x4.w, a);
+                }
+                acc[m] = a;
+            }
         }
+    }
+}
+
+// stage `rows` activation rows of n values (global, consecutive rows n apart) into the
+// padded shared-memory layout
+template <int FMT>
+__device__ __forceinline__ void stage_padded(float* dst, const float* src, int rows, int n, bool stream)
+{
+    constexpr int pc = Fmt<FMT>::per_chunk;
+    const int n4 = n / 4, total = rows * n4;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int r = i / n4, c4 = i - r * n4, col = 4 * c4;
+        const float4 v = stream ? __ldcg(reinterpret_cast<const float4*>(src) + i)
+                                : __ldg(reinterpret_cast<const float4*>(src) + i);
+        *reinterpret_cast<float4*>(dst + (size_t)r * padded_row<FMT>(n) + (col / pc) * Fmt<FMT>::pad_chunk + col % pc) = v;
     }
 }
 
@@ -123,10 +159,9 @@ __device__ __forceinline__ int seg_tokens(const FmtParams& p, int seg, int (&tok
 template <int FMT>
 __global__ void __launch_bounds__(kFmtThreads) fmt_gate_up_kernel(const __grid_constant__ FmtParams p)
 {
-    extern __shared__ __align__(16) float xs[];   // [T][H]
+    extern __shared__ __align__(16) float xs[];   // [T] padded rows of x
     const int H = p.H, I = p.I, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < p.T * H / 4; i += kFmtThreads)
-        reinterpret_cast<float4*>(xs)[i] = __ldg(reinterpret_cast<const float4*>(p.x) + i);
+    stage_padded<FMT>(xs, p.x, p.T, H, false);
     __syncthreads();
     const int nu = *reinterpret_cast<const volatile int32_t*>(p.n_union);
     const int nseg = p.n_shared + nu;
@@ -152,8 +187,8 @@ __global__ void __launch_bounds__(kFmtThreads) fmt_gate_up_kernel(const __grid_c
             const float sg = __half2float(gsc[Fmt<FMT>::per_row ? 0 : col / 64]);
             const float su = __half2float(usc[Fmt<FMT>::per_row ? 0 : col / 64]);
             float ag[kFmtMaxT] = {0.f, 0.f, 0.f, 0.f}, au[kFmtMaxT] = {0.f, 0.f, 0.f, 0.f};
-            chunk_dot<FMT>(gw, xs, H, col, cnt, tok, ag);
-            chunk_dot<FMT>(uw, xs, H, col, cnt, tok, au);
+            chunk_dot<FMT>(gw, xs, padded_row<FMT>(H), ch, cnt, tok, ag);
+            chunk_dot<FMT>(uw, xs, padded_row<FMT>(H), ch, cnt, tok, au);
 #pragma unroll
             for (int m = 0; m < kFmtMaxT; m++) {
                 g[m] = fmaf(ag[m], sg, g[m]);
@@ -171,7 +206,7 @@ __global__ void __launch_bounds__(kFmtThreads) fmt_gate_up_kernel(const __grid_c
 template <int FMT>
 __global__ void __launch_bounds__(kFmtThreads) fmt_down_kernel(const __grid_constant__ FmtParams p)
 {
-    extern __shared__ __align__(16) float hs[];   // [T][I]: one segment's h rows
+    extern __shared__ __align__(16) float hs[];   // one segment's h rows, padded
     const int H = p.H, I = p.I, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nu = *reinterpret_cast<const volatile int32_t*>(p.n_union);
     const int nseg = p.n_shared + nu;
@@ -190,8 +225,7 @@ __global__ void __launch_bounds__(kFmtThreads) fmt_down_kernel(const __grid_cons
         const uint8_t* blob;
         const int cnt = seg_tokens(p, seg, tok, wt, hbase, blob);
         __syncthreads();
-        for (int i = threadIdx.x; i < cnt * I / 4; i += kFmtThreads)
-            reinterpret_cast<float4*>(hs)[i] = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)hbase * I) + i);
+        stage_padded<FMT>(hs, p.h + (size_t)hbase * I, cnt, I, true);
         __syncthreads();
         int ident[kFmtMaxT];
 #pragma unroll
@@ -208,7 +242,7 @@ __global__ void __launch_bounds__(kFmtThreads) fmt_down_kernel(const __grid_cons
                 const int col = ch * Fmt<FMT>::per_chunk;
                 const float sd = __half2float(dsc[Fmt<FMT>::per_row ? 0 : col / 64]);
                 float a[kFmtMaxT] = {0.f, 0.f, 0.f, 0.f};
-                chunk_dot<FMT>(dw, hs, I, col, cnt, ident, a);
+                chunk_dot<FMT>(dw, hs, padded_row<FMT>(I), ch, cnt, ident, a);
 #pragma unroll
                 for (int m = 0; m < kFmtMaxT; m++) d[m] = fmaf(a[m], sd, d[m]);
             }
@@ -239,7 +273,7 @@ __global__ void __launch_bounds__(kFmtThreads) fmt_down_kernel(const __grid_cons
 template <int FMT>
 cudaError_t launch_fmt(const FmtParams& p, int num_sms, cudaStream_t s)
 {
-    const size_t sx = (size_t)p.T * p.H * 4, sh = (size_t)p.T * p.I * 4;
+    const size_t sx = (size_t)p.T * padded_row<FMT>(p.H) * 4, sh = (size_t)p.T * padded_row<FMT>(p.I) * 4;
     cudaError_t e = cudaFuncSetAttribute(fmt_gate_up_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sx);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fmt_down_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);

@@ -151,3 +151,26 @@ def test_per_row_equals_gs64_with_equal_group_scales():
                 FMT_INT4_ROW, *inputs(np.random.default_rng(9)))
     diff = np.nonzero((yr2 != yr).any(axis=0))[0]
     assert diff.tolist() == [7]
+
+
+@pytest.mark.parametrize("fmt", [FMT_INT4_G64, FMT_INT8_G64, FMT_INT4_ROW, FMT_INT2_G64])
+def test_quantizer_blob_decodes_to_its_dequantised_weights(fmt):
+    """The package's host quantiser packs what the oracle's decoder reads back: every
+    sampled weight of the blob equals the quantiser's dequantised value, and the rounding
+    error is at most half a step (inside the code range)."""
+    from int4_routed_expert_gemv_b200 import quantize as Q
+    rng = np.random.default_rng(30 + fmt)
+    G = (rng.standard_normal((I, H)) * 0.05).astype(np.float32)
+    U = (rng.standard_normal((I, H)) * 0.05).astype(np.float32)
+    D = (rng.standard_normal((H, I)) * 0.05).astype(np.float32)
+    blob_q, (Gd, Ud, Dd) = Q.expert_blob(G, U, D, fmt)
+    assert blob_q.size == oracle.blob_bytes_fmt(H, I, fmt)
+    for which, M, Md in [(0, G, Gd), (1, U, Ud), (2, D, Dd)]:
+        rows, cols = M.shape
+        for r, c in zip(rng.integers(0, rows, 40), rng.integers(0, cols, 40)):
+            assert oracle.blob_weight_fmt(H, I, fmt, blob_q, which, int(r), int(c)) == float(Md[r, c])
+        q, s = Q.quantize_matrix(M, fmt)
+        step = np.repeat(s.astype(np.float32), cols // s.shape[1], axis=1)
+        lo, hi = Q.QRANGE[fmt]
+        inside = (M / step > lo - 0.5) & (M / step < hi + 0.5)
+        assert np.all(np.abs(M - Md)[inside] <= 0.5 * step[inside] * (1 + 1e-6))
