@@ -244,6 +244,21 @@ COLI_API coli_status coli_moe_forward_fmt(const coli_moe_dims* dims, int32_t fmt
                                           const int32_t* assign, const float* residual, float* y,
                                           void* ws, size_t ws_bytes, void* stream);
 
+/* Expert parallelism (experts split over ranks in contiguous id ranges; README.zh-CN
+ * "实际成果", the technical article's "集群模式与开放问题清单"): the entries of a batch union
+ * (from coli_moe_union / coli_moe_route_union over all E experts) whose experts lie in
+ * [e0, e1), renumbered to e - e0: union_ids_local [e1-e0] (ascending, then -1),
+ * n_union_local (device int32), offsets_local [e1-e0+1], assign_local [T*k] (positions
+ * t*k+slot into the full idx / w arrays, first offsets_local[n_union_local] of them
+ * valid).  Passing these lists, the rank's experts (stride as usual, expert e0 first), the
+ * full w, and dims with n_experts = e1-e0 to coli_moe_forward gives the rank's share of
+ * y; the shares of all ranks (the shared expert counted on one rank only) add up to y. */
+COLI_API coli_status coli_moe_union_restrict(const coli_moe_dims* dims, int32_t T, int32_t e0, int32_t e1,
+                                             const int32_t* union_ids, const int32_t* n_union,
+                                             const int32_t* offsets, const int32_t* assign,
+                                             int32_t* union_ids_local, int32_t* n_union_local,
+                                             int32_t* offsets_local, int32_t* assign_local, void* stream);
+
 /* Diagnostic: run one bounded device wait that can only run out (an mbarrier nothing
  * arrives at), with a budget of `budget_cycles` SM clock cycles (1 .. 2^32).  When the
  * budget is spent the kernel records COLI_DEV_TIMEOUT and timeout site 99 in the workspace

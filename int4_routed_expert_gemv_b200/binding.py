@@ -27,7 +27,7 @@ EXPORTS = [
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
     "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_moe_stack", "coli_rmsnorm",
     "coli_moe_forward_noalloc", "coli_moe_noalloc_read_status", "coli_debug_wait_timeout",
-    "coli_moe_blob_bytes_fmt", "coli_moe_forward_fmt",
+    "coli_moe_blob_bytes_fmt", "coli_moe_forward_fmt", "coli_moe_union_restrict",
     "coli_status_string",
 ]
 
@@ -83,6 +83,7 @@ def lib():
                 "coli_moe_noalloc_read_status": (i32, [ctypes.POINTER(ctypes.c_uint32), P]),
                 "coli_debug_wait_timeout": (i32, [P, sz, ctypes.c_uint64, P, P]),
                 "coli_moe_blob_bytes_fmt": (sz, [i32, i32, i32]),
+                "coli_moe_union_restrict": (i32, [D, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
                 "coli_moe_forward_fmt": (i32, [D, i32, W, P, i32, P, P, P, P, P, P, P, P, sz, P]),
                 "coli_status_string": (ctypes.c_char_p, [i32]),
             }
@@ -155,6 +156,13 @@ def coli_moe_forward_fmt(dims, fmt, weights, x, T, w, union_ids, n_union, offset
     return lib().coli_moe_forward_fmt(ctypes.byref(dims), int(fmt), ctypes.byref(weights), _p(x), T, _p(w),
                                       _p(union_ids), _p(n_union), _p(offsets), _p(assign), _p(residual), _p(y),
                                       _p(ws), ws.numel(), _s(stream))
+
+
+def coli_moe_union_restrict(dims, T, e0, e1, union_ids, n_union, offsets, assign, union_ids_l, n_union_l,
+                            offsets_l, assign_l, stream=None) -> int:
+    return lib().coli_moe_union_restrict(ctypes.byref(dims), T, e0, e1, _p(union_ids), _p(n_union), _p(offsets),
+                                         _p(assign), _p(union_ids_l), _p(n_union_l), _p(offsets_l), _p(assign_l),
+                                         _s(stream))
 
 
 def coli_moe_noalloc_read_status(stream=None):
