@@ -115,6 +115,9 @@ KERNEL_SOURCES = {
     "route_union": ["int4_routed_expert_gemv_b200/csrc/route.cu",
                     "int4_routed_expert_gemv_b200/csrc/select.cuh",
                     "int4_routed_expert_gemv_b200/csrc/union.cuh"],
+    "fused_moe_kernel": ["int4_routed_expert_gemv_b200/csrc/fused.cu",
+                         "int4_routed_expert_gemv_b200/csrc/fused.cuh",
+                         "int4_routed_expert_gemv_b200/csrc/common.cuh"],
 }
 
 
