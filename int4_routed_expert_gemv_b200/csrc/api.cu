@@ -21,7 +21,7 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t cnt, logits, h, xd, rpart, hf, xbuf, xchunk, gemm, total;
+    size_t cnt, logits, h, xd, rpart, hf, hdg, xbuf, xchunk, gemm, total;
 };
 
 constexpr size_t kCntBytes = (size_t)kCntWords * 4;
@@ -57,6 +57,8 @@ WsLayout ws_layout(const coli_moe_dims* d, int64_t T)
     off += (size_t)Tf * d->n_experts * (d->hidden / 128 > 0 ? d->hidden / 128 : 1) * 16;
     L.hf = off = up(off, kAlign);   // SwiGLU activations as (value, epoch) pairs
     off += (size_t)Tf * (d->top_k + d->n_shared) * d->inter * 8;
+    L.hdg = off = up(off, kAlign);  // one token: digit rows of h
+    off += (size_t)(d->top_k + d->n_shared) * hdg_row_bytes(d->inter);
     L.xbuf = off = up(off, kAlign);
     off += 2 * (size_t)Tf * d->hidden * sizeof(float);
     L.xchunk = off = up(off, kAlign);
@@ -188,6 +190,8 @@ bool fused_setup(FusedParams& f, const coli_moe_dims* d, int32_t T, int L, void*
     f.cnt = reinterpret_cast<uint32_t*>(base + W.cnt);
     f.rpart = reinterpret_cast<uint4*>(base + W.rpart);
     f.h = reinterpret_cast<uint2*>(base + W.hf);
+    f.hdg = base + W.hdg;
+    f.hdg_row = (uint32_t)hdg_row_bytes(d->inter);
     f.xbuf = reinterpret_cast<float*>(base + W.xbuf);
     return true;
 }

@@ -112,6 +112,13 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return pol;
 }
 
+// Orders this thread's earlier generic-proxy accesses to global memory (and what they
+// observed) before its later asynchronous-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes,
                                          uint64_t* bar)
 {

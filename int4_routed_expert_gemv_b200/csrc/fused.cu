@@ -60,6 +60,8 @@ constexpr float kPf0 = 1.0f / 16.0f;
 constexpr float kPf1 = 1.0f / (16.0f * 254.0f);
 constexpr float kPf2 = 1.0f / (16.0f * 254.0f * 254.0f);
 
+constexpr int kDigBufs = 4;   // pair mode: digit rows of h in flight per CTA
+
 struct Head {
     uint64_t full[kMaxSlots];
     uint64_t empty[kMaxSlots];
@@ -68,6 +70,8 @@ struct Head {
     uint32_t gen;                // launch generation (h epochs)
     uint64_t red_full[8];        // partial-sum buffer b: every consumer warp delivered
     uint64_t red_empty[8];       // partial-sum buffer b: summed, free again
+    uint64_t dg_full[kDigBufs];  // pair mode: digit row buffer b filled (one bulk copy)
+    uint64_t dg_empty[kDigBufs]; // pair mode: every consumer warp has read buffer b
     double rsq[NCW][kFusedMaxT];
     double rnorm[kFusedMaxT];
     float amax[NCW][kFusedMaxT];
@@ -262,8 +266,8 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 // 64-column group, 16-31 the second).  Each value becomes three balanced int8 digits of
 // X = x * 126 / m (m = the group's largest magnitude): X ~ a + b/254 + c/254^2, |error| <=
 // 0.5/254^2 + rounding, a in [-126, 126], b, c in [-127, 127].  The lane's three plane
-// words (4 digits each, column order) go to sc[plane * 32 + l]; returns m of its group.
-__device__ __forceinline__ float digits128(float4 v, int lane, uint32_t* sc)
+// words (4 digits each, column order) go to wd[plane]; returns m of its group.
+__device__ __forceinline__ float digit_words(float4 v, uint32_t (&wd)[3])
 {
     float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -283,9 +287,20 @@ __device__ __forceinline__ float digits128(float4 v, int lane, uint32_t* sc)
         const float e2 = (e1 - bf) * 254.0f;
         dc[i] = rint_small(e2, cf);
     }
-    sc[lane] = pack4(da[0], da[1], da[2], da[3]);
-    sc[32 + lane] = pack4(db[0], db[1], db[2], db[3]);
-    sc[64 + lane] = pack4(dc[0], dc[1], dc[2], dc[3]);
+    wd[0] = pack4(da[0], da[1], da[2], da[3]);
+    wd[1] = pack4(db[0], db[1], db[2], db[3]);
+    wd[2] = pack4(dc[0], dc[1], dc[2], dc[3]);
+    return mx;
+}
+
+// digit_words with the lane's three plane words stored to sc[plane * 32 + lane].
+__device__ __forceinline__ float digits128(float4 v, int lane, uint32_t* sc)
+{
+    uint32_t wd[3];
+    const float mx = digit_words(v, wd);
+    sc[lane] = wd[0];
+    sc[32 + lane] = wd[1];
+    sc[64 + lane] = wd[2];
     return mx;
 }
 
@@ -621,52 +636,10 @@ __device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, 
     }
 }
 
-// Digits of one token's h row (I columns), once per CTA: warp w digitizes group pairs w,
-// w + NCW, ... into the compact buffer dig (plane p: I bytes at p * I, column order) and the
-// group factors m / 126 into fac.  (value, epoch) pairs are read until they carry `epoch`.
-__device__ __forceinline__ void digitize_h_row(const uint2* staged, const uint2* row, uint32_t epoch, int I,
-                                               int warp, int lane, uint32_t* sc, uint32_t* dig, float* fac,
-                                               uint32_t* status, volatile int* dead)
-{
-    const int npairs = I / 128;
-#pragma unroll 1
-    for (int pp = warp; pp < npairs; pp += NCW) {
-        // the staged copy first; where it holds another epoch's values (the copy ran before
-        // the producer's store), poll the row itself
-        const uint4* sp = reinterpret_cast<const uint4*>(staged + 128 * pp + 4 * lane);
-        uint4 a = sp[0], b = sp[1];
-        bool ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
-        if (!ok) {
-            const uint4* hp = reinterpret_cast<const uint4*>(row + 128 * pp + 4 * lane);
-            const long long t0 = clock64();
-            uint32_t npoll = 0;
-            while (true) {
-                a = __ldcg(hp);
-                b = __ldcg(hp + 1);
-                ok = __all_sync(0xffffffffu, a.y == epoch && a.w == epoch && b.y == epoch && b.w == epoch);
-                if (ok) break;
-                if (*dead || wait_expired(npoll, t0, status)) {
-                    if (lane == 0) give_up(status, 56, dead);
-                    break;
-                }
-                __nanosleep(128);
-            }
-        }
-        const float4 v = make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x),
-                                     __uint_as_float(b.z));
-        const float mx = digits128(v, lane, sc);
-        __syncwarp();
-#pragma unroll
-        for (int pl = 0; pl < 3; pl++) dig[pl * (I / 4) + 32 * pp + lane] = sc[pl * 32 + lane];
-        if (lane == 0) fac[2 * pp] = mx * (1.0f / 126.0f);
-        if (lane == 16) fac[2 * pp + 1] = mx * (1.0f / 126.0f);
-        __syncwarp();
-    }
-}
-
-// Pair-form operand of the warp's groups from the compact digits of digitize_h_row.
+// Pair-form operand of the warp's groups from a digit row (planes of I bytes, then the
+// (m / 126, epoch) words of the groups).
 template <int GPWM, int NTM>
-__device__ __forceinline__ void gather_h_pairs(const uint32_t* dig, const float* facs, int I, int gbase,
+__device__ __forceinline__ void gather_h_pairs(const uint32_t* dig, const uint2* tags, int I, int gbase,
                                                int lane, uint32_t (&B)[GPWM][NTM][4],
                                                float (&fac)[GPWM][NTM])
 {
@@ -690,7 +663,7 @@ __device__ __forceinline__ void gather_h_pairs(const uint32_t* dig, const float*
         r[7] = __byte_perm(w1.z, w1.w, 0x7531);
 #pragma unroll
         for (int i = 0; i < 8; i++) B[2 * pi + (i >> 2)][0][i & 3] = r[i] & keep;
-        fac[2 * pi][0] = facs[gbase + 2 * pi + (tq >> 1)];
+        fac[2 * pi][0] = __uint_as_float(tags[gbase + 2 * pi + (tq >> 1)].x);
         fac[2 * pi + 1][0] = 0.0f;
     }
 }
@@ -1040,6 +1013,7 @@ __device__ __forceinline__ uint32_t h_epoch(const Ctx& c, int l)
 struct Stream {
     uint32_t it;
     uint64_t pol;
+    uint32_t dd;   // pair mode: digit rows copied so far (every down segment)
 };
 
 __device__ __forceinline__ uint8_t* slot_begin(const FusedParams& p, const Ctx& c, Stream& st,
@@ -1103,6 +1077,42 @@ __device__ __forceinline__ void issue_down(const FusedParams& p, const Ctx& c, S
                           bar, st.pol);
     }
     bulk_g2s_hint(dst + p.d_sc_off, blob + c.bo.ds + a0, (uint32_t)(a1 - a0), bar, st.pol);
+}
+
+// One token: the digit row of h row `row` (layer l) into digit buffer dd % kDigBufs, once
+// every consumer warp has released the buffer and every group of the row carries the
+// layer's epoch (bounded polls), as one bulk copy completing on the buffer's barrier.
+__device__ __forceinline__ void issue_digits(const FusedParams& p, const Ctx& c, Stream& st, int l, int row)
+{
+    const int lane = c.lane, I = p.I, ng = I / 64;
+    const uint32_t b = st.dd % (uint32_t)kDigBufs;
+    if (st.dd >= (uint32_t)kDigBufs)
+        mwait(&c.hd->dg_empty[b], ((st.dd / (uint32_t)kDigBufs) - 1u) & 1u, p.status, 33, c.dead);
+    const uint8_t* src = p.hdg + (size_t)row * p.hdg_row;
+    const unsigned long long* tags = reinterpret_cast<const unsigned long long*>(src + 3 * (size_t)I);
+    const uint32_t ep = __ldcg(p.gen) * 32u + (uint32_t)l + 1u;
+    const long long t0 = clock64();
+    uint32_t npoll = 0;
+    while (true) {
+        bool ok = true;
+#pragma unroll 1
+        for (int g = lane; g < ng; g += 32) ok = ok && (uint32_t)(__ldcg(tags + g) >> 32) == ep;
+        if (__all_sync(0xffffffffu, ok)) break;
+        if (*c.dead || wait_expired(npoll, t0, p.status)) {
+            if (lane == 0) give_up(p.status, 34, c.dead);
+            break;
+        }
+        __nanosleep(64);
+    }
+    __threadfence();
+    fence_proxy_async_global();
+    if (lane == 0) {
+        uint64_t* bar = &c.hd->dg_full[b];
+        mbar_arrive_expect_tx(bar, p.hdg_row);
+        bulk_g2s(reinterpret_cast<uint8_t*>(c.hd) + p.off_hdig + (size_t)b * p.hdig_bytes, src, p.hdg_row, bar);
+    }
+    st.dd++;
+    __syncwarp();
 }
 
 // ----------------------------- control warp: routing ------------------------------------
@@ -1309,6 +1319,7 @@ __device__ __forceinline__ void control_warp(const FusedParams& p, const Ctx& c)
 {
     Stream st;
     st.it = 0;
+    st.dd = 0;
     st.pol = policy_evict_first();
     const int ns = p.n_shared;
 #pragma unroll 1
@@ -1332,6 +1343,7 @@ __device__ __forceinline__ void control_warp(const FusedParams& p, const Ctx& c)
                 nseg = tb.hdr[0];
                 routed = true;
             } else if (c.nrows > 0 && ds < nseg) {
+                if (p.pair) issue_digits(p, c, st, l, ds < ns ? p.T * p.k : tb.base[ds]);
                 if (c.lane == 0)
                     issue_down(p, c, st, ds < ns ? ly.shared : ly.experts + (uint64_t)tb.e[ds] * ly.stride);
                 ds++;
@@ -1367,22 +1379,6 @@ struct Cons {
     int g_rs, g_kw, gbase_g, gpw_g;   // gate/up: row slot, K slot, its groups
     int d_rs, d_kw, gbase_d, gpw_d;   // down
 };
-
-// One token's h row `base` (I values with their epochs) into staging buffer buf & 1 by
-// asynchronous copies (each warp the 128-value pieces it digitizes), as one commit group.
-__device__ __forceinline__ void h_prefetch(const FusedParams& p, const Ctx& c, int base, uint32_t buf)
-{
-    const int I = p.I;
-    const uint2* row = reinterpret_cast<const uint2*>(p.h) + (size_t)base * I;
-    uint2* stg = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_hstage + (size_t)(buf & 1u) * 8u * I);
-#pragma unroll 1
-    for (int pp = c.warp; pp < I / 128; pp += NCW) {
-        const int o = 128 * pp + 4 * c.lane;
-        cp_async16(stg + o, row + o);
-        cp_async16(stg + o + 2, row + o + 2);
-    }
-    cp_async_commit();
-}
 
 __device__ __forceinline__ const uint8_t* cslot_wait(const FusedParams& p, const Ctx& c, Cons& w)
 {
@@ -1696,7 +1692,7 @@ __device__ __forceinline__ void gu_consume(const FusedParams& p, const Ctx& c, C
 // the down stage of segment s (this CTA's output rows), combined into yacc
 template <int NTM, int GPWD, bool PAIR>
 __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c, Cons& w, int l,
-                                             const Seg& sg, int next_base, uint32_t (&Bh)[GPWD][NTM][4],
+                                             const Seg& sg, uint32_t (&Bh)[GPWD][NTM][4],
                                              float (&fh)[GPWD][NTM])
 {
     const int T = p.T, I = p.I, lane = c.lane;
@@ -1704,24 +1700,15 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
     const uint32_t ep = h_epoch(c, l);
     const uint2* hb = reinterpret_cast<const uint2*>(p.h);
     if constexpr (PAIR) {
-        // the segment's h digits once per CTA (double-buffered), then each warp's operand.
-        // h arrives by asynchronous copies issued one segment ahead (staging buffer
-        // ds & 1); the next segment's copies are issued before this one's are awaited
-        uint8_t* hd0 = reinterpret_cast<uint8_t*>(c.hd) + p.off_hdig + (size_t)(w.ds & 1) * p.hdig_bytes;
-        uint32_t* dig = reinterpret_cast<uint32_t*>(hd0);
-        float* facs = reinterpret_cast<float*>(hd0 + 3 * I);
-        if (next_base >= 0) {
-            h_prefetch(p, c, next_base, w.ds + 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
+        // the segment's digit row of h, copied by the control warp into buffer ds % kDigBufs
+        // (the ds-th down segment of the launch); the buffer is released once read
+        const uint32_t ds = w.ds, b = ds % (uint32_t)kDigBufs;
+        const uint8_t* hd0 = reinterpret_cast<const uint8_t*>(c.hd) + p.off_hdig + (size_t)b * p.hdig_bytes;
+        mwait(&c.hd->dg_full[b], (ds / (uint32_t)kDigBufs) & 1u, p.status, 58, c.dead);
+        gather_h_pairs<GPWD, NTM>(reinterpret_cast<const uint32_t*>(hd0), reinterpret_cast<const uint2*>(hd0 + 3 * I),
+                                  I, w.gbase_d, lane, Bh, fh);
         __syncwarp();
-        const uint2* stg = reinterpret_cast<const uint2*>(reinterpret_cast<uint8_t*>(c.hd) + p.off_hstage +
-                                                          (size_t)(w.ds & 1) * 8u * I);
-        digitize_h_row(stg, hb + (size_t)sg.base * I, ep, I, c.warp, lane, w.sc, dig, facs, p.status, c.dead);
-        named_bar(6, NCT);
-        gather_h_pairs<GPWD, NTM>(dig, facs, I, w.gbase_d, lane, Bh, fh);
+        if (lane == 0) mbar_arrive(&c.hd->dg_empty[b]);
         w.ds++;
     } else {
 #pragma unroll
@@ -1770,8 +1757,86 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
 // ----------------------------- reducer warp ---------------------------------------------
 // Sums of one gate/up stage (stage st of segment sg): four lanes per (row, token) over the
 // K-split warps' partials, SwiGLU, h stored as (value, epoch).
+// One token: the digit rows of h.  Group g (64 values) of h row `row` is digitized by
+// one CTA (the one that sums the group's last row) once all its values carry the layer's
+// epoch; lane j (and j + 16) holds values 64 g + 4 j .. + 3 as (value, epoch) pairs.
+__device__ __forceinline__ void group_load(const FusedParams& p, int row, int g, int lane, uint4& a, uint4& b)
+{
+    const uint4* hp = reinterpret_cast<const uint4*>(p.h + (size_t)row * p.I + 64 * g + 4 * (lane & 15));
+    a = __ldcg(hp);
+    b = __ldcg(hp + 1);
+}
+
+__device__ __forceinline__ bool group_ready(const uint4& a, const uint4& b, uint32_t ep)
+{
+    return __all_sync(0xffffffffu, a.y == ep && a.w == ep && b.y == ep && b.w == ep);
+}
+
+// The group's digits into the row's digit row, then its (m / 126, ep) word, ordered after
+// the digits (a reader that sees the word sees the digits).
+__device__ __forceinline__ void group_store(const FusedParams& p, int row, int g, int lane, uint32_t ep,
+                                            const uint4& a, const uint4& b)
+{
+    const int I = p.I;
+    uint32_t wd[3];
+    const float m = digit_words(make_float4(__uint_as_float(a.x), __uint_as_float(a.z), __uint_as_float(b.x),
+                                            __uint_as_float(b.z)), wd);
+    uint8_t* dr = p.hdg + (size_t)row * p.hdg_row;
+    if (lane < 16) {
+#pragma unroll
+        for (int pl = 0; pl < 3; pl++)
+            *reinterpret_cast<uint32_t*>(dr + (size_t)pl * I + 64 * g + 4 * lane) = wd[pl];
+    }
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence();
+        *reinterpret_cast<unsigned long long*>(dr + 3 * (size_t)I + 8 * g) =
+            ((unsigned long long)ep << 32) | __float_as_uint(m * (1.0f / 126.0f));
+    }
+}
+
+// The groups this CTA still has to digitize, oldest first (lane j holds entry j:
+// row << 16 | group).
+struct Pending {
+    uint32_t e;
+    int n;
+};
+
+__device__ __forceinline__ void pending_pop(Pending& pd)
+{
+    pd.e = __shfl_down_sync(0xffffffffu, pd.e, 1);
+    pd.n--;
+}
+
+// Every pending group, each once its values have arrived (bounded waits).
+__device__ __forceinline__ void pending_drain(const FusedParams& p, const Ctx& c, Pending& pd, uint32_t ep)
+{
+#pragma unroll 1
+    while (pd.n > 0) {
+        const uint32_t e0 = __shfl_sync(0xffffffffu, pd.e, 0);
+        const int row = (int)(e0 >> 16), g = (int)(e0 & 0xFFFFu);
+        uint4 a, b;
+        group_load(p, row, g, c.lane, a, b);
+        if (!group_ready(a, b, ep)) {
+            const long long t0 = clock64();
+            uint32_t npoll = 0;
+            while (true) {
+                __nanosleep(64);
+                group_load(p, row, g, c.lane, a, b);
+                if (group_ready(a, b, ep)) break;
+                if (*c.dead || wait_expired(npoll, t0, p.status)) {
+                    if (c.lane == 0) give_up(p.status, 56, c.dead);
+                    break;
+                }
+            }
+        }
+        group_store(p, row, g, c.lane, ep, a, b);
+        pending_pop(pd);
+    }
+}
+
 __device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, uint32_t cs, const Seg& sg,
-                                          int st, uint32_t ep)
+                                          int st, uint32_t ep, Pending& pd)
 {
     const int T = p.T, I = p.I, lane = c.lane;
     const float* rb = c.red + (size_t)(cs % kRedBufs) * p.red_floats;
@@ -1805,30 +1870,48 @@ __device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, ui
             hb[(size_t)(sg.base + m) * I + row] = make_uint2(__float_as_uint(hv), ep);
         }
     }
+    if (p.pair) {
+        // one token: this CTA digitizes every group whose last row is one of the stage's
+        // rows i0 .. i0 + 8 ntl - 1, once all its values have arrived
+        const int r1 = i0 + 8 * ntl;
+#pragma unroll 1
+        for (int g = i0 / 64; g <= (r1 - 1) / 64; g++) {
+            if (64 * g + 63 < i0 || 64 * g + 63 >= r1) continue;
+            if (pd.n == 32) pending_drain(p, c, pd, ep);
+            if (lane == pd.n) pd.e = ((uint32_t)sg.base << 16) | (uint32_t)g;
+            pd.n++;
+        }
+    }
 }
 
 // Sums of one down stage (segment sg, the CTA's rows): routing-weighted combine into yacc.
+// One lane per (row, token); the K-split partials kw are added as ((s0 + s1) + (s2 + s3)),
+// s_j the sum of those with kw = j mod 4 in ascending kw.
 __device__ __forceinline__ void reduce_down(const FusedParams& p, const Ctx& c, uint32_t cs, const Seg& sg)
 {
-    const int T = p.T, lane = c.lane, cn = sg.c, ntdm = p.ntdm;
+    const int T = p.T, lane = c.lane, cn = sg.c, KW = p.KWd;
     const float* rb = c.red + (size_t)(cs % kRedBufs) * p.red_floats;
-    const int ntask = c.ntd * 16 * cn, part = lane & 3;
+    const int nrs = c.ntd * 16;                        // row slots of the CTA's tiles
+    const size_t kst = (size_t)p.ntdm * 16 * T;        // from one K-split warp's part to the next
 #pragma unroll 1
-    for (int t0 = 0; t0 < ntask; t0 += 8) {
-        const int task = t0 + (lane >> 2);
-        const int m = task % cn, rr = task / cn;
-        const int tl = rr >> 4, mm = rr & 15;
-        const int q = mm & 3, lrow = 4 * tl + (mm >> 2);
-        const bool valid = task < ntask && lrow < dcs(c, q + 1) - dcs(c, q);
-        float sum = 0.0f;
-        if (valid)
+    for (int m = 0; m < cn; m++) {
+        const float wt = sg.wt[m];
+        const int tok = sg.tok[m];
 #pragma unroll 1
-            for (int kw = part; kw < p.KWd; kw += 4) sum += rb[((size_t)(kw * ntdm + tl) * 16 + mm) * T + m];
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (valid && part == 0) {
-            float* ya = c.yacc + (dcs(c, q) + lrow) * T + sg.tok[m];
-            *ya = *ya + sg.wt[m] * sum;
+        for (int rr = lane; rr < nrs; rr += 32) {
+            const int tl = rr >> 4, mm = rr & 15;
+            const int q = mm & 3, lrow = 4 * tl + (mm >> 2);
+            if (lrow >= dcs(c, q + 1) - dcs(c, q)) continue;
+            const float* src = rb + ((size_t)tl * 16 + mm) * T + m;
+            float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+            for (int k0 = 0; k0 < KW; k0 += 4) {
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    if (k0 + j < KW) s4[j] += src[(size_t)(k0 + j) * kst];
+            }
+            float* ya = c.yacc + (dcs(c, q) + lrow) * T + tok;
+            *ya = *ya + wt * ((s4[0] + s4[1]) + (s4[2] + s4[3]));
         }
     }
 }
@@ -1844,6 +1927,9 @@ __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c,
     sh.tok = c.hd->sh_tok;
     sh.wt = c.hd->sh_wt;
     uint32_t cs = 0;
+    Pending pd;
+    pd.e = 0u;
+    pd.n = 0;
 #pragma unroll 1
     for (int l = 0; l < p.L; l++) {
         const uint32_t ep = gen * 32u + (uint32_t)l + 1u;
@@ -1867,10 +1953,21 @@ __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c,
             } else {
                 break;
             }
+            // the groups of h left to digitize, before the first down stage (every CTA's
+            // down stages need them); otherwise the oldest one's values are read while the
+            // partial sums are awaited, and it is digitized after the stage if they are all in
+            if (kind == 2 && pd.n > 0) pending_drain(p, c, pd, ep);
+            const bool look = pd.n > 0;
+            uint4 ga = make_uint4(0u, 0u, 0u, 0u), gb = ga;
+            uint32_t ge = 0u;
+            if (look) {
+                ge = __shfl_sync(0xffffffffu, pd.e, 0);
+                group_load(p, (int)(ge >> 16), (int)(ge & 0xFFFFu), lane, ga, gb);
+            }
             mwait(&c.hd->red_full[cs % kRedBufs], (cs / kRedBufs) & 1u, p.status, 59, c.dead);
             const Seg sg = seg < ns ? sh : seg_of(tb, seg);
             if (kind == 1) {
-                reduce_gu(p, c, cs, sg, gi - seg * p.SPS, ep);
+                reduce_gu(p, c, cs, sg, gi - seg * p.SPS, ep, pd);
                 gi += c.G;
             } else {
                 reduce_down(p, c, cs, sg);
@@ -1878,7 +1975,13 @@ __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c,
             __syncwarp();
             if (lane == 0) mbar_arrive(&c.hd->red_empty[cs % kRedBufs]);
             cs++;
+            if (look && group_ready(ga, gb, ep)) {
+                group_store(p, (int)(ge >> 16), (int)(ge & 0xFFFFu), lane, ep, ga, gb);
+                pending_pop(pd);
+            }
         }
+        // (a CTA without down rows still digitizes its groups)
+        if (pd.n > 0) pending_drain(p, c, pd, ep);
         // the layer's output rows are summed: the consumers write them, then yacc is clear
         named_bar(7, NCT + 32);
         named_bar(8, NCT + 32);
@@ -1978,10 +2081,6 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                     gi += c.G;
                 } else {
                     phase = 6;
-                    // the first down segment's h on its way into shared memory
-                    if constexpr (PAIR)
-                        if (c.nrows > 0 && nseg > 0)
-                            h_prefetch(p, c, ns ? sh.base : seg_of(tb, 0).base, w.ds);
                     continue;
                 }
             } else {
@@ -1999,14 +2098,12 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                 if (kind == 1) {
                     gu_consume<NTM, GPWG, PAIR>(p, c, w, l, sg, stage, Bx, fdummy);
                 } else {
-                    // the base row of the next down segment's h (prefetched), or -1
-                    const int nb = sd < nseg ? (sd < ns ? sh.base : seg_of(tb, sd).base) : -1;
                     if constexpr (GPWG == GPWD) {
                         // the h operand takes the x operand's registers (the down stages
                         // follow every gate/up stage of the layer)
-                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, nb, Bx, fdummy);
+                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bx, fdummy);
                     } else {
-                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, nb, Bh, fh);
+                        down_consume<NTM, GPWD, PAIR>(p, c, w, l, sg, Bh, fh);
                     }
                 }
             }
@@ -2071,6 +2168,11 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
             mbar_init(&c.hd->red_empty[b2], 1);
         }
 #pragma unroll 1
+        for (int b2 = 0; b2 < kDigBufs; b2++) {
+            mbar_init(&c.hd->dg_full[b2], 1);
+            mbar_init(&c.hd->dg_empty[b2], NCW);
+        }
+#pragma unroll 1
         for (int m = 0; m < kFusedMaxT; m++) {
             c.hd->sh_tok[m] = m;
             c.hd->sh_wt[m] = 1.0f;
@@ -2102,6 +2204,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
             __threadfence();
 #pragma unroll 1
             for (int i = 1; i < 1 + p.L * kCntPerLayer; i++) p.cnt[i] = 0u;
+
             *p.gen = c.hd->gen + 1u;
             __threadfence();
             p.cnt[0] = 0u;
@@ -2202,7 +2305,7 @@ bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
     // one token: both matrices in group pairs when each splits into warp shares of exactly 4
     // or 8 aligned groups; the 16-byte row reads need the chunks 64 bytes (mod 128) apart
     p.pair = 0;
-    if (T == 1 && H % 512 == 0 && I % 512 == 0 && H <= 16 * NCT) {
+    if (T == 1 && H % 512 == 0 && I % 512 == 0 && H <= 16 * NCT && p.k + p.n_shared <= 65535) {
         const int kg = kw_pair(ngg), kd = kw_pair(ngd);
         if (kg && kd) {
             p.pair = 1;
@@ -2264,12 +2367,11 @@ bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
     off = up128(off + (uint32_t)kRedBufs * p.red_floats * 4u);
     p.off_yacc = off;
     off = up128(off + (uint32_t)p.rows_max * T * 4u);
-    p.hdig_bytes = p.pair ? (uint32_t)(3 * I + 4 * (I / 64)) : 0u;
+    p.hdig_bytes = p.pair ? up128((uint32_t)hdg_row_bytes(I)) : 0u;
     p.off_hdig = off;
-    off = up128(off + 2u * p.hdig_bytes);
-    p.off_hstage = off;   // pair mode: two staged h rows (value, epoch)
-    // (the same area holds the layer input row before the down stages)
-    off = up128(off + (p.pair ? (2u * 8u * (uint32_t)I > 4u * (uint32_t)H ? 2u * 8u * (uint32_t)I : 4u * (uint32_t)H) : 0u));
+    off = up128(off + (uint32_t)kDigBufs * p.hdig_bytes);
+    p.off_hstage = off;   // pair mode: the layer input row
+    off = up128(off + (p.pair ? 4u * (uint32_t)H : 0u));
     p.off_scratch = off;
     // consumer digit scratch (96 words per warp), then the control warp's logits,
     // selections, weights and bitmaps

@@ -20,6 +20,13 @@ constexpr int kFusedMaxSeg = 1 + kFusedMaxT * kFusedMaxK;   // shared expert + u
 constexpr int kCntPerLayer = 2 + kFusedMaxSeg;
 constexpr int kCntWords = 1 + kFusedMaxLayers * kCntPerLayer;
 
+// Bytes of one digit row of h (I values): three planes of I digit bytes, then one
+// (m / 126, epoch) word pair per 64-value group; a multiple of 16.
+__host__ __device__ constexpr size_t hdg_row_bytes(int I)
+{
+    return ((size_t)(3 * I + 8 * (I / 64)) + 15) / 16 * 16;
+}
+
 struct FusedLayer {
     const float* w_router;   // [E][H]
     const float* bias;       // [E] or null
@@ -58,6 +65,9 @@ struct FusedParams {
     uint32_t* cnt;           // kCntWords counters, zero between launches
     uint4* rpart;            // [T][E][RC] router partial sums: (low word, epoch, high word, epoch)
     uint2* h;                // [T*(k+n_shared)][I] SwiGLU activations as (value, epoch)
+    uint8_t* hdg;            // one token: per h row its digit row (3 planes of I bytes, then
+                             // (m / 126, epoch) per 64-value group), hdg_row bytes apart
+    uint32_t hdg_row;
     // plan (fused_plan)
     int grid, nslot;
     uint32_t slot_bytes;
@@ -72,8 +82,8 @@ struct FusedParams {
     uint32_t gu_chunk, gu_gsc, gu_usc;   // gate/up stage: chunk stride, scale areas
     uint32_t d_chunk, d_sc_off;          // down stage: chunk stride, scale area
     uint32_t red_floats;                 // one partial-sum buffer
-    uint32_t off_hdig, hdig_bytes;       // pair mode: compact h digits, two buffers
-    uint32_t off_hstage;                 // pair mode: two staged h rows
+    uint32_t off_hdig, hdig_bytes;       // pair mode: kDigBufs copies of digit rows
+    uint32_t off_hstage;                 // pair mode: the layer input row
     uint32_t off_red, off_yacc, off_scratch, off_ring;   // dynamic shared memory layout
 };
 
