@@ -137,6 +137,13 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p)
     return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -1096,7 +1103,7 @@ __device__ __forceinline__ void issue_digits(const FusedParams& p, const Ctx& c,
     while (true) {
         bool ok = true;
 #pragma unroll 1
-        for (int g = lane; g < ng; g += 32) ok = ok && (uint32_t)(__ldcg(tags + g) >> 32) == ep;
+        for (int g = lane; g < ng; g += 32) ok = ok && (uint32_t)(ld_acquire64(tags + g) >> 32) == ep;
         if (__all_sync(0xffffffffu, ok)) break;
         if (*c.dead || wait_expired(npoll, t0, p.status)) {
             if (lane == 0) give_up(p.status, 34, c.dead);
@@ -1104,7 +1111,9 @@ __device__ __forceinline__ void issue_digits(const FusedParams& p, const Ctx& c,
         }
         __nanosleep(64);
     }
-    __threadfence();
+    // each lane's tag reads acquire the digits written before them; the warp barrier
+    // orders them before lane 0's copy, which the proxy fence orders after the reads
+    __syncwarp();
     fence_proxy_async_global();
     if (lane == 0) {
         uint64_t* bar = &c.hd->dg_full[b];
