@@ -1504,6 +1504,7 @@ __device__ __forceinline__ void load_x_pair(const FusedParams& p, const Ctx& c, 
         const int u = tid + NCT * j;
         v[j] = u < n4 ? __ldcg(reinterpret_cast<const float4*>(xin) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    if (tid == 0) hd.gen = __ldcg(p.gen);   // published by the named barriers below
     double r = 1.0;
     if (p.norm) {
         double sq = 0.0;
@@ -2200,7 +2201,9 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
         reducer_warp(p, c, __ldcg(p.gen));
     } else {
         pdl_wait();
-        if (c.tid == 0) c.hd->gen = __ldcg(p.gen);   // published by the first named barrier
+        // the launch generation, published by the first named barrier (one token: read in
+        // load_x_pair beside the layer input, so the two loads overlap)
+        if (!PAIR && c.tid == 0) c.hd->gen = __ldcg(p.gen);
         consumer_warp<NTM, GPWG, GPWD, PAIR>(p, c);
     }
 
