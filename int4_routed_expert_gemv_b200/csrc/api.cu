@@ -217,9 +217,13 @@ coli_status run_gemv(int mode, GemvParams& p, cudaStream_t s)
 
 bool gemv_shape_ok(const coli_moe_dims* d, int32_t T)
 {
+    // the current device's SM count and shared memory; without a usable device the B200's
+    // (the call then fails at its first CUDA step with COLI_ECUDA)
     DevInfo di;
-    di.sms = 148;
-    di.smem_optin = 232448;
+    if (!dev_info(di)) {
+        di.sms = 148;
+        di.smem_optin = 232448;
+    }
     for (int mode = 0; mode < 2; mode++) {
         GemvParams p;
         memset(&p, 0, sizeof(p));
