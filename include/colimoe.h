@@ -267,6 +267,20 @@ COLI_API coli_status coli_moe_union_restrict(const coli_moe_dims* dims, int32_t 
 COLI_API coli_status coli_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t budget_cycles,
                                              int32_t* returned, void* stream);
 
+/* Diagnostic: the phase stamps of the last fused decode launch (coli_moe_layer /
+ * coli_moe_stack for 1-4 tokens), for a library built with COLI_PHASE_STAMPS
+ * (`python -m int4_routed_expert_gemv_b200.build --stamps`; the phase table of
+ * `python -m int4_routed_expert_gemv_b200.phases`).  Copies, for up to max_ctas CTAs,
+ * *n_stamps (16) global-timer values in ns per CTA into the host array stamps
+ * [max_ctas][16]: 0 kernel entry, 1 layer input loaded, 2 router partial sums published,
+ * 3 input operand built, 4 routing table ready, 5 first routed gate/up stage, 6 first down
+ * stage, 7 last down stage done, 8 last reduction done, 9 exit (the last layer of the
+ * launch; 0 where a CTA has no such phase, and rows of all 0 beyond the launch's
+ * CTAs).  Synchronises with the device.  Returns
+ * COLI_EUNSUPPORTED (and *n_stamps = 0) for the regular build. */
+COLI_API coli_status coli_debug_phase_stamps(uint64_t* stamps, int32_t max_ctas, int32_t* n_ctas,
+                                             int32_t* n_stamps);
+
 /* Residual stack of decode layers, every layer resident in device memory:
  *   for l in 0 .. n_layers-1:  n = RMSNorm_l(x);  x = x + MoE_l(n);   y = x at the end,
  * with RMSNorm_l(x) = x * gamma[l] / sqrt(mean(x^2) + eps) (double, rounded once to fp32)

@@ -27,6 +27,7 @@ EXPORTS = [
     "coli_moe_read_status", "coli_moe_route", "coli_moe_route_union", "coli_moe_union", "coli_moe_forward",
     "coli_moe_gate_up", "coli_moe_down", "coli_moe_layer", "coli_moe_stack", "coli_rmsnorm",
     "coli_moe_forward_noalloc", "coli_moe_noalloc_read_status", "coli_debug_wait_timeout",
+    "coli_debug_phase_stamps",
     "coli_moe_blob_bytes_fmt", "coli_moe_forward_fmt", "coli_moe_union_restrict",
     "coli_status_string",
 ]
@@ -82,6 +83,7 @@ def lib():
                 "coli_moe_forward_noalloc": (i32, [D, W, P, i32, P, P, P, P, P, P, P, P]),
                 "coli_moe_noalloc_read_status": (i32, [ctypes.POINTER(ctypes.c_uint32), P]),
                 "coli_debug_wait_timeout": (i32, [P, sz, ctypes.c_uint64, P, P]),
+                "coli_debug_phase_stamps": (i32, [P, i32, P, P]),
                 "coli_moe_blob_bytes_fmt": (sz, [i32, i32, i32]),
                 "coli_moe_union_restrict": (i32, [D, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
                 "coli_moe_forward_fmt": (i32, [D, i32, W, P, i32, P, P, P, P, P, P, P, P, sz, P]),
@@ -173,6 +175,15 @@ def coli_moe_noalloc_read_status(stream=None):
 
 def coli_debug_wait_timeout(ws: torch.Tensor, budget_cycles: int, returned: torch.Tensor, stream=None) -> int:
     return lib().coli_debug_wait_timeout(_p(ws), ws.numel(), int(budget_cycles), _p(returned), _s(stream))
+
+
+def coli_debug_phase_stamps(max_ctas: int = 256):
+    """(status, stamps [n_ctas][n_stamps] as a numpy uint64 array) of the last fused launch."""
+    import numpy as np
+    buf = np.zeros((max_ctas, 16), np.uint64)
+    n_ctas, n_st = ctypes.c_int32(0), ctypes.c_int32(0)
+    st = lib().coli_debug_phase_stamps(buf.ctypes.data, max_ctas, ctypes.byref(n_ctas), ctypes.byref(n_st))
+    return st, buf[:n_ctas.value, :n_st.value]
 
 
 def coli_moe_read_status(ws: torch.Tensor, stream=None):

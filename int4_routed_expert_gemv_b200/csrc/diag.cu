@@ -50,3 +50,22 @@ extern "C" coli_status coli_debug_wait_timeout(void* ws, size_t ws_bytes, uint64
                                                            returned);
     return cudaGetLastError() == cudaSuccess ? COLI_OK : COLI_ECUDA;
 }
+
+namespace coli {
+int fused_phase_stamps(unsigned long long* host, int max_ctas, int* n_stamps);
+}
+
+// Phase stamps of the last fused launch (a library built with COLI_PHASE_STAMPS; the
+// regular build returns COLI_EUNSUPPORTED).
+extern "C" coli_status coli_debug_phase_stamps(uint64_t* stamps, int32_t max_ctas, int32_t* n_ctas,
+                                              int32_t* n_stamps)
+{
+    if (!stamps || !n_ctas || !n_stamps || max_ctas < 1) return COLI_EINVAL;
+    int ns = 0;
+    const int n = coli::fused_phase_stamps(reinterpret_cast<unsigned long long*>(stamps), max_ctas, &ns);
+    if (n < 0) return COLI_ECUDA;
+    *n_ctas = n;
+    *n_stamps = ns;
+    return ns == 0 ? COLI_EUNSUPPORTED : COLI_OK;
+}
+

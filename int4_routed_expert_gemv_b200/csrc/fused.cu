@@ -62,6 +62,39 @@ constexpr float kPf2 = 1.0f / (16.0f * 254.0f * 254.0f);
 
 constexpr int kDigBufs = 4;   // pair mode: digit rows of h in flight per CTA
 
+// Phase stamps (builds with COLI_PHASE_STAMPS only; compiled out otherwise): one thread
+// per CTA writes the global nanosecond timer at the phase boundaries of the launch's last
+// layer, stamp i of CTA b at g_phase[b * kStamps + i].
+constexpr int kStamps = 16;
+constexpr int kStampCtas = 256;
+enum : int {
+    ST_START = 0,        // kernel entry
+    ST_INPUT = 1,        // consumers: layer input loaded, scales formed
+    ST_ROUTER = 2,       // consumers: router partial sums published
+    ST_XOP = 3,          // consumers: input operand built
+    ST_TABLE = 4,        // control warp: routing table ready
+    ST_GU_ROUTED = 5,    // consumers: first routed gate/up stage begins
+    ST_DOWN = 6,         // consumers: first down stage begins
+    ST_DOWN_DONE = 7,    // consumers: last down stage done
+    ST_REDUCED = 8,      // reducer: last reduction done
+    ST_EXIT = 9,         // kernel exit
+};
+#ifdef COLI_PHASE_STAMPS
+__device__ unsigned long long g_phase[kStampCtas * kStamps];
+__device__ __forceinline__ void stamp(bool on, int i)
+{
+    if (on && blockIdx.x < kStampCtas) {
+        if (i == ST_START)   // the CTA's row of the previous launch is cleared first
+            for (int j = 1; j < kStamps; j++) g_phase[blockIdx.x * kStamps + j] = 0ull;
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        g_phase[blockIdx.x * kStamps + i] = t;
+    }
+}
+#else
+__device__ __forceinline__ void stamp(bool, int) {}
+#endif
+
 struct Head {
     uint64_t full[kMaxSlots];
     uint64_t empty[kMaxSlots];
@@ -1349,6 +1382,7 @@ __device__ __forceinline__ void control_warp(const FusedParams& p, const Ctx& c)
                 __syncwarp();
                 if (l == 0) pdl_wait();
                 route_layer(p, c, l, l == 0);
+                stamp(c.lane == 0 && l == p.L - 1, ST_TABLE);
                 nseg = tb.hdr[0];
                 routed = true;
             } else if (c.nrows > 0 && ds < nseg) {
@@ -1992,6 +2026,7 @@ __device__ __forceinline__ void reducer_warp(const FusedParams& p, const Ctx& c,
         }
         // (a CTA without down rows still digitizes its groups)
         if (pd.n > 0) pending_drain(p, c, pd, ep);
+        stamp(lane == 0 && l == p.L - 1, ST_REDUCED);
         // the layer's output rows are summed: the consumers write them, then yacc is clear
         named_bar(7, NCT + 32);
         named_bar(8, NCT + 32);
@@ -2043,9 +2078,12 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
         }
         // the router needs only the RMSNorm factors (1 for a plain input), so for a plain
         // input it runs first and the routing is decided while the scales are formed
+        const bool w0 = c.warp == 0 && c.lane == 0 && l == p.L - 1;
         if constexpr (PAIR) {
             load_x_pair(p, c, l, xin);
+            stamp(w0, ST_INPUT);
             if (c.ri1 > c.ri0) router_consume<true>(p, c, w, l, xin);
+            stamp(w0, ST_ROUTER);
         } else {
 #pragma unroll 1
             for (int step = 0; step < 2; step++) {
@@ -2055,12 +2093,15 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                     input_scales(p, c, l, xin);
                 }
             }
+            stamp(w0, ST_INPUT);
+            stamp(w0, ST_ROUTER);
         }
         // stages in the control warp's order; one code path per kind of step
         //   phase 0: x operand, 1: shared gate/up, 4: routing, 5: routed gate/up,
         //   6: down rows of every segment (the shared expert's first)
         Table tb;
         int nseg = 0, phase = 0, gi = c.b, sd = 0;
+        bool routed_seen = false;   // phase stamps: a routed gate/up stage has begun
         while (true) {
             int kind = -1, seg = 0, stage = 0;   // 0: x operand, 1: gate/up, 2: down
             if (phase == 0) {
@@ -2103,11 +2144,15 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
             }
             if (kind == 0) {
                 build_x_operand<NTM, GPWG, PAIR>(p, c, w, l, xin, Bx, fdummy);
+                stamp(w0, ST_XOP);
             } else {
                 const Seg sg = seg < ns ? sh : seg_of(tb, seg);
                 if (kind == 1) {
+                    stamp(w0 && seg >= ns && !routed_seen, ST_GU_ROUTED);
+                    routed_seen = routed_seen || seg >= ns;
                     gu_consume<NTM, GPWG, PAIR>(p, c, w, l, sg, stage, Bx, fdummy);
                 } else {
+                    stamp(w0 && seg == 0, ST_DOWN);
                     if constexpr (GPWG == GPWD) {
                         // the h operand takes the x operand's registers (the down stages
                         // follow every gate/up stage of the layer)
@@ -2118,6 +2163,7 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
                 }
             }
         }
+        stamp(w0, ST_DOWN_DONE);
         // ---- this CTA's rows of the layer output (once the reducer has summed them all)
         named_bar(7, NCT + 32);
 #pragma unroll 1
@@ -2164,6 +2210,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
     c.bo = blob_off(p.H, p.I);
 
     pdl_launch_dependents();
+    stamp(c.tid == 0, ST_START);
     if (c.tid == 0) {
 #pragma unroll 1
         for (int s = 0; s < p.nslot; s++) {
@@ -2209,6 +2256,7 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
 
     // ---- exit: the last CTA returns the counters to zero and advances the generation
     __syncthreads();
+    stamp(c.tid == 0, ST_EXIT);
     if (c.tid == 0) {
         __threadfence();
         const uint32_t prev = atomicAdd(&p.cnt[0], 1u);
@@ -2281,6 +2329,22 @@ inline int kw_pair(int n)
 constexpr int kGpwMax = 8;
 
 }  // namespace
+
+int fused_phase_stamps(unsigned long long* host, int max_ctas, int* n_stamps)
+{
+#ifdef COLI_PHASE_STAMPS
+    *n_stamps = kStamps;
+    const int n = max_ctas < kStampCtas ? max_ctas : kStampCtas;
+    if (cudaMemcpyFromSymbol(host, g_phase, sizeof(unsigned long long) * (size_t)n * kStamps) != cudaSuccess)
+        return -1;
+    return n;
+#else
+    (void)host;
+    (void)max_ctas;
+    *n_stamps = 0;
+    return 0;
+#endif
+}
 
 bool fused_plan(FusedParams& p, int num_sms, size_t smem_limit)
 {
