@@ -2262,11 +2262,11 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
         const uint32_t prev = atomicAdd(&p.cnt[0], 1u);
         if (prev == (uint32_t)c.G - 1u) {
             __threadfence();
+            // the only counter a layer uses is its output-rows count; the next launch, which
+            // follows this one in stream order, sees these stores without a further fence
 #pragma unroll 1
-            for (int i = 1; i < 1 + p.L * kCntPerLayer; i++) p.cnt[i] = 0u;
-
+            for (int l = 0; l < p.L; l++) layer_cnt(p, l)[1] = 0u;
             *p.gen = c.hd->gen + 1u;
-            __threadfence();
             p.cnt[0] = 0u;
         }
     }
