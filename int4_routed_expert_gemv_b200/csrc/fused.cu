@@ -2175,7 +2175,8 @@ __device__ __forceinline__ void consumer_warp(const FusedParams& p, const Ctx& c
             c.yacc[i] = 0.0f;
         }
         named_bar(8, NCT + 32);
-        if (c.tid == 0) {
+        // the next layer's consumers wait for every CTA's rows (none wait after the last)
+        if (c.tid == 0 && l < p.L - 1) {
             __threadfence();
             red_release_add(&lc[1], 1u);
         }
@@ -2257,13 +2258,13 @@ __global__ void __launch_bounds__(NTHR, 1) fused_moe_kernel(const __grid_constan
     // ---- exit: the last CTA returns the counters to zero and advances the generation
     __syncthreads();
     stamp(c.tid == 0, ST_EXIT);
+    // (every layer's output-rows increments were seen by the waits of the layer after it,
+    // so the counters the last CTA clears are no longer written by anyone)
     if (c.tid == 0) {
-        __threadfence();
         const uint32_t prev = atomicAdd(&p.cnt[0], 1u);
         if (prev == (uint32_t)c.G - 1u) {
-            __threadfence();
             // the only counter a layer uses is its output-rows count; the next launch, which
-            // follows this one in stream order, sees these stores without a further fence
+            // follows this one in stream order, sees these stores without a fence
 #pragma unroll 1
             for (int l = 0; l < p.L; l++) layer_cnt(p, l)[1] = 0u;
             *p.gen = c.hd->gen + 1u;
