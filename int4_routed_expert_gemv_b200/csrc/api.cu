@@ -57,8 +57,8 @@ WsLayout ws_layout(const coli_moe_dims* d, int64_t T)
     off += (size_t)Tf * d->n_experts * (d->hidden / 128 > 0 ? d->hidden / 128 : 1) * 16;
     L.hf = off = up(off, kAlign);   // SwiGLU activations as (value, epoch) pairs
     off += (size_t)Tf * (d->top_k + d->n_shared) * d->inter * 8;
-    L.hdg = off = up(off, kAlign);  // one token: digit rows of h
-    off += (size_t)(d->top_k + d->n_shared) * hdg_row_bytes(d->inter);
+    L.hdg = off = up(off, kAlign);  // digit rows of h (one per row of hf)
+    off += (size_t)Tf * (d->top_k + d->n_shared) * hdg_row_bytes(d->inter);
     L.xbuf = off = up(off, kAlign);
     off += 2 * (size_t)Tf * d->hidden * sizeof(float);
     L.xchunk = off = up(off, kAlign);

@@ -676,6 +676,59 @@ __device__ __forceinline__ void build_h_pairs(const uint2* row, uint32_t epoch, 
     }
 }
 
+// Two-token column tile q of the warp's groups (as build_tile lays them out: lanes 16-31
+// token slot 1, lane groups by digit plane, per-group factors by threadID >> 1) from the
+// digit rows of h in global memory (drow0 / drow1 for the tile's tokens, absent when !p0 /
+// !p1).  Every group's (m / 126, epoch) word is read until it carries `epoch` (bounded),
+// acquiring the digits written before it; then the digit words are loaded.
+template <int GPWM, int NTM>
+__device__ __forceinline__ void gather_tile_digits(const uint8_t* drow0, const uint8_t* drow1, bool p0, bool p1,
+                                                   int I, uint32_t epoch, int gbase, int gpw, int q, int lane,
+                                                   uint32_t (&B)[GPWM][NTM][4], float (&fac)[GPWM][NTM],
+                                                   uint32_t* status, volatile int* dead)
+{
+    const int bslot = lane >> 4, plane = (lane >> 2) & 3, tq = lane & 3, fslot = tq >> 1;
+    const int pl = plane < 3 ? plane : 0;
+    const uint32_t keep = plane < 3 ? 0xFFFFFFFFu : 0u;
+    // lane j < 2 gpw checks the word of token slot j / gpw, group j % gpw
+    {
+        const int js = lane / (gpw > 0 ? gpw : 1), jg = lane - js * gpw;
+        const bool mine = lane < 2 * gpw && (js ? p1 : p0);
+        const unsigned long long* tag = reinterpret_cast<const unsigned long long*>(
+            (js ? drow1 : drow0) + 3 * (size_t)I + 8 * (size_t)(gbase + jg));
+        const long long t0 = clock64();
+        uint32_t npoll = 0;
+        while (true) {
+            const bool ok = !mine || (uint32_t)(ld_acquire64(tag) >> 32) == epoch;
+            if (__all_sync(0xffffffffu, ok)) break;
+            if (*dead || wait_expired(npoll, t0, status)) {
+                if (lane == 0) give_up(status, 56, dead);
+                break;
+            }
+            __nanosleep(64);
+        }
+        __syncwarp();
+    }
+    const bool pb = bslot ? p1 : p0, pf = fslot ? p1 : p0;
+    const uint8_t* rb = bslot ? drow1 : drow0;
+    const uint8_t* rf = fslot ? drow1 : drow0;
+#pragma unroll
+    for (int gi = 0; gi < GPWM; gi++) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        float f = 0.0f;
+        if (gi < gpw) {
+            if (pb) w = __ldcg(reinterpret_cast<const uint4*>(rb + (size_t)pl * I + 64 * (gbase + gi) + 16 * tq));
+            if (pf) f = __uint_as_float(__ldcg(reinterpret_cast<const unsigned int*>(rf + 3 * (size_t)I +
+                                                                                      8 * (size_t)(gbase + gi))));
+        }
+        B[gi][q][0] = __byte_perm(w.x, w.y, 0x6420) & keep;
+        B[gi][q][1] = __byte_perm(w.x, w.y, 0x7531) & keep;
+        B[gi][q][2] = __byte_perm(w.z, w.w, 0x6420) & keep;
+        B[gi][q][3] = __byte_perm(w.z, w.w, 0x7531) & keep;
+        fac[gi][q] = f;
+    }
+}
+
 // Pair-form operand of the warp's groups from a digit row (planes of I bytes, then the
 // (m / 126, epoch) words of the groups).
 template <int GPWM, int NTM>
@@ -1742,7 +1795,6 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
     const int T = p.T, I = p.I, lane = c.lane;
     const int cn = sg.c;
     const uint32_t ep = h_epoch(c, l);
-    const uint2* hb = reinterpret_cast<const uint2*>(p.h);
     if constexpr (PAIR) {
         // the segment's digit row of h, copied by the control warp into buffer ds % kDigBufs
         // (the ds-th down segment of the launch); the buffer is released once read
@@ -1759,10 +1811,10 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
         for (int q = 0; q < NTM; q++) {
             const int m0 = 2 * q, m1 = 2 * q + 1;
             const bool p0 = m0 < cn, p1 = m1 < cn;
-            const uint2* row0 = hb + (size_t)(sg.base + (p0 ? m0 : 0)) * I;
-            const uint2* row1 = hb + (size_t)(sg.base + (p1 ? m1 : 0)) * I;
-            build_tile<GPWD, NTM, true>(row0, row1, p0, p1, 0.f, 0.f, 1.0, 1.0, nullptr, ep,
-                                        w.gbase_d, w.gpw_d, q, w.sc, lane, Bh, fh, p.status, c.dead);
+            const uint8_t* d0 = p.hdg + (size_t)(sg.base + (p0 ? m0 : 0)) * p.hdg_row;
+            const uint8_t* d1 = p.hdg + (size_t)(sg.base + (p1 ? m1 : 0)) * p.hdg_row;
+            gather_tile_digits<GPWD, NTM>(d0, d1, p0, p1, I, ep, w.gbase_d, w.gpw_d, q, lane, Bh, fh, p.status,
+                                          c.dead);
         }
     }
     const uint32_t qmask = (1u << ((cn + 1) >> 1)) - 1u;
@@ -1914,16 +1966,19 @@ __device__ __forceinline__ void reduce_gu(const FusedParams& p, const Ctx& c, ui
             hb[(size_t)(sg.base + m) * I + row] = make_uint2(__float_as_uint(hv), ep);
         }
     }
-    if (p.pair) {
-        // one token: this CTA digitizes every group whose last row is one of the stage's
-        // rows i0 .. i0 + 8 ntl - 1, once all its values have arrived
+    {
+        // this CTA digitizes, for each token of the segment, every group whose last row is
+        // one of the stage's rows i0 .. i0 + 8 ntl - 1, once all its values have arrived
         const int r1 = i0 + 8 * ntl;
 #pragma unroll 1
-        for (int g = i0 / 64; g <= (r1 - 1) / 64; g++) {
-            if (64 * g + 63 < i0 || 64 * g + 63 >= r1) continue;
-            if (pd.n == 32) pending_drain(p, c, pd, ep);
-            if (lane == pd.n) pd.e = ((uint32_t)sg.base << 16) | (uint32_t)g;
-            pd.n++;
+        for (int m = 0; m < sg.c; m++) {
+#pragma unroll 1
+            for (int g = i0 / 64; g <= (r1 - 1) / 64; g++) {
+                if (64 * g + 63 < i0 || 64 * g + 63 >= r1) continue;
+                if (pd.n == 32) pending_drain(p, c, pd, ep);
+                if (lane == pd.n) pd.e = ((uint32_t)(sg.base + m) << 16) | (uint32_t)g;
+                pd.n++;
+            }
         }
     }
 }
