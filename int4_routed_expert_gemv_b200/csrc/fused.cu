@@ -1853,7 +1853,7 @@ __device__ __forceinline__ void down_consume(const FusedParams& p, const Ctx& c,
 // ----------------------------- reducer warp ---------------------------------------------
 // Sums of one gate/up stage (stage st of segment sg): four lanes per (row, token) over the
 // K-split warps' partials, SwiGLU, h stored as (value, epoch).
-// One token: the digit rows of h.  Group g (64 values) of h row `row` is digitized by
+// The digit rows of h (one per row of h).  Group g (64 values) of h row `row` is digitized by
 // one CTA (the one that sums the group's last row) once all its values carry the layer's
 // epoch; lane j (and j + 16) holds values 64 g + 4 j .. + 3 as (value, epoch) pairs.
 __device__ __forceinline__ void group_load(const FusedParams& p, int row, int g, int lane, uint4& a, uint4& b)

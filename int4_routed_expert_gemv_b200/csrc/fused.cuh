@@ -65,7 +65,7 @@ struct FusedParams {
     uint32_t* cnt;           // kCntWords counters, zero between launches
     uint4* rpart;            // [T][E][RC] router partial sums: (low word, epoch, high word, epoch)
     uint2* h;                // [T*(k+n_shared)][I] SwiGLU activations as (value, epoch)
-    uint8_t* hdg;            // one token: per h row its digit row (3 planes of I bytes, then
+    uint8_t* hdg;            // per h row its digit row (3 planes of I bytes, then
                              // (m / 126, epoch) per 64-value group), hdg_row bytes apart
     uint32_t hdg_row;
     // plan (fused_plan)
